@@ -1,0 +1,171 @@
+/*
+ * matq.h -- C ABI of libmatq: sliced r-bit ("Matryoshka") linear layers on B200 (sm_100a).
+ *
+ * A weight matrix W [N, K] (torch.nn.Linear layout: N outputs, K inputs, K contiguous)
+ * is stored as ONE set of unsigned 8-bit parent codes q in [0, 255] with one fp16 scale s
+ * and one unsigned 8-bit zero point z per group of `group` consecutive inputs of a row.
+ * The scale and zero point are shared by every width ("Matryoshka Quantization | Summary",
+ * §3.1 MinMax quantizer; MatQuant rebuttal page, S.P. MatQuant item 2; "MatGPTQ: Efficient
+ * and Accurate Inference over Nested Quantized Models" §1, single shared-scale format).
+ *
+ * A width-r model, r in {2, 3, 4, 6, 8}, uses only the r most significant bits of every
+ * code (true-prefix slicing, MatGPTQ App. A.1):
+ *
+ *     p       = q >> (8 - r)                         (the prefix, 0 <= p < 2^r)
+ *     q_hat   = p * 2^(8-r) + delta_r,   delta_r = (2^(8-r) - 1) / 2
+ *     W_hat   = s * (q_hat - z)
+ *     y[m, n] = sum_k x[m, k] * W_hat[n, k]         (MatGPTQ §4: Y = X W_D)
+ *
+ * delta_r centres the value in its cell (App. A.1) and is folded into the zero point
+ * inside the kernels; a width-r call reads exactly r bits per weight (MatGPTQ §4).
+ *
+ * Conventions for every entry point
+ *   - All data pointers are caller-owned DEVICE memory unless stated; the library never
+ *     allocates, frees or keeps pointers between calls.
+ *   - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is asynchronous
+ *     on that stream; a returned MATQ_OK means "validated and launched", not "finished".
+ *   - Every call returns an int status: MATQ_OK (0) or a negative MATQ_E* code.  Argument
+ *     errors are caught on the host before any launch and leave every buffer untouched.
+ *     A launch failure returns MATQ_ECUDA; matq_last_cuda_error() gives the cudaError_t.
+ *   - Shapes: N >= 1; K a positive multiple of 256; M >= 1.  group in {64, 128}.
+ *   - Alignment: every device pointer must be 16-byte aligned.
+ *   - Thread safety: calls on different streams may run concurrently; the only state is a
+ *     thread-local "last CUDA error".
+ *
+ * Packed plane layout ("MATQ-PL1"; written by matq_pack, read by every other call)
+ *   The 8 code bits are split into five planes, most significant first:
+ *       plane 0: bits 7..6 (2 bits/weight)   plane 1: bit 5      plane 2: bit 4
+ *       plane 3: bits 3..2 (2 bits/weight)   plane 4: bits 1..0
+ *   Width r reads planes 0..P(r)-1 with P(2)=1, P(3)=2, P(4)=3, P(6)=4, P(8)=5; the bits of
+ *   those planes sum to r.  (The split into {1-2, 3, 4, 5-6, 7-8} MSB planes follows
+ *   MatGPTQ §4; the order of bits inside a plane is this library's own.)
+ *   Planes are stored back to back, plane 0 first, so the first matq_packed_bytes(N, K, r)
+ *   bytes of any pack with r_keep >= r are themselves a valid width-r pack ("mode A":
+ *   keep only the r-bit prefix resident; "mode B": keep all 8 bits and pass r per call).
+ *   Inside a plane of b bits/weight (b = 1 or 2) the matrix is cut into row tiles of 16 rows
+ *   (RT = ceil(N/16); rows >= N are packed as code 0) and K-chunks of 256 inputs
+ *   (KC = K/256).  Tile (rt, kc) occupies b*512 bytes at byte offset (rt*KC + kc)*b*512.
+ *   Inside a tile, the 4096 weights are dealt to 32 "lanes" (lane = 4*gid + tg, gid in 0..7,
+ *   tg in 0..3), 128 weights each, in the operand order of a 16x16 fp16 MMA tile:
+ *     block w in 0..7 covers inputs 32w..32w+31 of the chunk; in block w a lane holds 16
+ *     fields f = 0..15 with u = f & 7, hi = f >> 3, j = u >> 2, rho = u & 3 and
+ *         row = 16*rt + gid + 8*(rho & 1)
+ *         k   = 256*kc + 32*w + 16*j + 2*tg + 8*(rho >> 1) + hi.
+ *   2-bit planes: lane word w (w = 0..7) holds field f of block w in bits [2f, 2f+2); the
+ *     tile is two 512-byte halves: words 0..3 of all lanes (lane-major, 16 bytes a lane),
+ *     then words 4..7.
+ *   1-bit planes: lane word v (v = 0..3) holds blocks 2v + a (a = 0, 1), field f of block
+ *     2v + a at bit 4*(f >> 1) + 2*a + (f & 1); the tile is 32 lanes x 16 bytes.
+ *   So a warp streams each plane with 16-byte-per-lane coalesced loads, and a lane's words
+ *   turn into MMA operand registers with a few shifts and masks.
+ */
+#ifndef MATQ_H
+#define MATQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------------------ */
+#define MATQ_OK             0
+#define MATQ_EINVAL_R      -1   /* r not in {2,3,4,6,8}, or r > r_keep is MATQ_ETRUNC     */
+#define MATQ_EINVAL_SHAPE  -2   /* N < 1, M < 1, K < 256 or K % 256 != 0, overflow          */
+#define MATQ_EINVAL_GROUP  -3   /* group not in {64, 128}                                   */
+#define MATQ_EALIGN        -4   /* a device pointer is not 16-byte aligned                  */
+#define MATQ_ENULL         -5   /* a required pointer is NULL                               */
+#define MATQ_ETRUNC        -6   /* the pack holds fewer planes than width r needs           */
+#define MATQ_ECUDA         -7   /* a CUDA call or launch failed: see matq_last_cuda_error   */
+#define MATQ_ESIZE         -8   /* a caller buffer (planes, workspace) is too small          */
+#define MATQ_EDTYPE        -9   /* unknown output mode                                      */
+#define MATQ_EDEVICE      -10   /* current device is not sm_100 (B200 class)               */
+
+/* ---- output modes of matq_linear ----------------------------------------------------- */
+#define MATQ_OUT_BF16       0   /* y [M, N] bf16 = x . W_hat^T                             */
+#define MATQ_OUT_F32        1   /* y [M, N] fp32 = x . W_hat^T                             */
+#define MATQ_OUT_F32_ACCUM  2   /* y [M, N] fp32 += x . W_hat^T (fused residual add)       */
+
+/* Library version (major*10000 + minor*100 + patch). */
+int matq_version(void);
+
+/* Human-readable text of a status code (static storage, never NULL). */
+const char* matq_strerror(int status);
+
+/* cudaError_t of the last failing CUDA call made by this thread (0 if none). */
+int matq_last_cuda_error(void);
+
+/* ---- layout queries (host only, no CUDA call) ---------------------------------------- */
+
+/* Number of planes width r reads: 1, 2, 3, 4, 5 for r = 2, 3, 4, 6, 8; 0 if r is invalid. */
+int matq_plane_count(int r);
+
+/* Bytes of planes needed to serve every width <= r_keep:
+ *     ceil(N/16) * 16 * K * r_keep / 8     (exactly r_keep bits per weight when 16 | N).
+ * Returns 0 on invalid arguments (N < 1, K % 256 != 0, r_keep not a valid width). */
+size_t matq_packed_bytes(int N, int K, int r_keep);
+
+/* ---- one-time pack (§ "efficient packing", MatGPTQ §1 contribution 3 and §4) ---------- */
+
+/* Repack parent codes into the MATQ-PL1 plane layout, keeping the planes of widths
+ * <= r_keep.
+ *   codes        [N, K] uint8, row-major, device.  Read only.
+ *   planes       device buffer of at least matq_packed_bytes(N, K, r_keep) bytes; written.
+ *   planes_bytes capacity of `planes` (MATQ_ESIZE if too small).
+ * Every code byte is read once and every plane bit written once. */
+int matq_pack(const uint8_t* codes, int N, int K, int r_keep,
+              void* planes, size_t planes_bytes, void* stream);
+
+/* Recover the width-r prefixes p = q >> (8 - r) from a pack (verification and export).
+ *   planes     pack written with r_keep >= r (MATQ_ETRUNC otherwise).
+ *   prefix_out [N, K] uint8, row-major, device; written. */
+int matq_slice(const void* planes, int N, int K, int r_keep, int r,
+               uint8_t* prefix_out, void* stream);
+
+/* Deployment mode A: copy the width-r prefix of a pack (its first matq_packed_bytes(N,K,r)
+ * bytes) into `planes_r`, which then is a width-r pack (r_keep = r) on its own.
+ *   bytes  capacity of planes_r (MATQ_ESIZE if < matq_packed_bytes(N, K, r)). */
+int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r,
+                    void* planes_r, size_t bytes, void* stream);
+
+/* ---- the sliced linear layer ----------------------------------------------------------- */
+
+/* Workspace bytes matq_linear needs for these sizes (a multiple of 256). */
+size_t matq_linear_workspace(int M, int K, int N, int group);
+
+/* y = x . W_hat_r^T for a width-r slice of a pack.
+ *   x        [M, K] bf16, row-major, device.  Read only.
+ *   planes   pack with r_keep >= r.  Read only; exactly the planes of width r are read.
+ *   scales   [N, K/group] fp16 (raw bits), row-major.  zeros [N, K/group] uint8.
+ *   y        [M, N] row-major, dtype by y_mode (MATQ_OUT_*).  MATQ_OUT_F32_ACCUM adds the
+ *            product to the fp32 values already in y.
+ *   workspace device scratch of >= matq_linear_workspace(M, K, N, group) bytes, owned by
+ *            the caller; its contents need no initialisation and are clobbered.  Calls that
+ *            share a workspace must be ordered (same stream, or synchronised).
+ * Kernel choice is internal: M <= 16 takes the decode path (warp-level streaming GEMV /
+ * skinny GEMM, fp32 accumulation); larger M the prefill path (TMA-staged planes,
+ * dequantised to fp16 tiles in shared memory, tcgen05 MMA with TMEM accumulators).
+ * The prefill path rounds x and W_hat to fp16; it needs |x| and |W_hat| below 65504. */
+int matq_linear(const void* x, int M, int K,
+                const void* planes, int r_keep,
+                const uint16_t* scales, const uint8_t* zeros, int N,
+                int r, int group,
+                void* y, int y_mode,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- glue of the Mix'n'Match FFN stack ------------------------------------------------- */
+
+/* n = bf16( h / sqrt(mean(h^2) + eps) ) row by row (unit-gain RMSNorm).
+ *   h [M, D] fp32, n_out [M, D] bf16. */
+int matq_rmsnorm(const float* h, int M, int D, float eps, void* n_out, void* stream);
+
+/* a = bf16( silu(gate) * up ), silu(t) = t / (1 + exp(-t)), computed in fp32.
+ *   gate, up, a_out [M, F] bf16. */
+int matq_silu_mul(const void* gate, const void* up, int M, int F, void* a_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MATQ_H */

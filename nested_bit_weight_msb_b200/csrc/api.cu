@@ -1,0 +1,167 @@
+// C ABI of libmatq (declared in include/matq.h): host-side validation and dispatch.
+// Every argument error is caught here, before any CUDA call, and returned as a status.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/matq.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace matq;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MATQ_OK;
+  g_last_cuda_error = (int)e;
+  return MATQ_ECUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool valid_nk(int N, int K) {
+  if (N < 1 || K < kChunk || K % kChunk != 0) return false;
+  // keep every byte offset and index comfortably inside 64-bit / int ranges
+  if ((long long)N * (long long)K > (1LL << 40)) return false;
+  if ((long long)((N + 15) / 16) * (K / kChunk) > (1LL << 31) - 1) return false;
+  return true;
+}
+
+int check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  int major = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  return major == 10 ? MATQ_OK : MATQ_EDEVICE;
+}
+
+size_t packed_bytes(int N, int K, int r_keep) {
+  const PlaneGeom g = make_geom(N, K);
+  size_t total = 0;
+  for (int p = 0; p < planes_for_width(r_keep); ++p) total += (size_t)plane_bytes(g.RT, g.KC, p);
+  return total;
+}
+
+}  // namespace
+
+extern "C" {
+
+int matq_version(void) { return 100; }
+
+const char* matq_strerror(int status) {
+  switch (status) {
+    case MATQ_OK: return "ok";
+    case MATQ_EINVAL_R: return "invalid width r (must be 2, 3, 4, 6 or 8)";
+    case MATQ_EINVAL_SHAPE: return "invalid shape (N >= 1, M >= 1, K a positive multiple of 256)";
+    case MATQ_EINVAL_GROUP: return "invalid group size (must be 64 or 128)";
+    case MATQ_EALIGN: return "device pointer not 16-byte aligned";
+    case MATQ_ENULL: return "required pointer is NULL";
+    case MATQ_ETRUNC: return "pack holds fewer planes than width r needs (r > r_keep)";
+    case MATQ_ECUDA: return "CUDA call failed (see matq_last_cuda_error)";
+    case MATQ_ESIZE: return "caller buffer too small";
+    case MATQ_EDTYPE: return "unknown output mode";
+    case MATQ_EDEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    default: return "unknown status";
+  }
+}
+
+int matq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int matq_plane_count(int r) { return planes_for_width(r); }
+
+size_t matq_packed_bytes(int N, int K, int r_keep) {
+  if (!valid_width(r_keep) || !valid_nk(N, K)) return 0;
+  return packed_bytes(N, K, r_keep);
+}
+
+int matq_pack(const uint8_t* codes, int N, int K, int r_keep, void* planes, size_t planes_bytes, void* stream) {
+  if (!valid_width(r_keep)) return MATQ_EINVAL_R;
+  if (!valid_nk(N, K)) return MATQ_EINVAL_SHAPE;
+  if (!codes || !planes) return MATQ_ENULL;
+  if (!aligned16(codes) || !aligned16(planes)) return MATQ_EALIGN;
+  if (planes_bytes < packed_bytes(N, K, r_keep)) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_pack(codes, make_geom(N, K), r_keep, planes, (cudaStream_t)stream));
+}
+
+int matq_slice(const void* planes, int N, int K, int r_keep, int r, uint8_t* prefix_out, void* stream) {
+  if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
+  if (r > r_keep) return MATQ_ETRUNC;
+  if (!valid_nk(N, K)) return MATQ_EINVAL_SHAPE;
+  if (!planes || !prefix_out) return MATQ_ENULL;
+  if (!aligned16(planes) || !aligned16(prefix_out)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_slice(planes, make_geom(N, K), r, prefix_out, (cudaStream_t)stream));
+}
+
+int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r, void* planes_r, size_t bytes,
+                    void* stream) {
+  if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
+  if (r > r_keep) return MATQ_ETRUNC;
+  if (!valid_nk(N, K)) return MATQ_EINVAL_SHAPE;
+  if (!planes || !planes_r) return MATQ_ENULL;
+  if (!aligned16(planes) || !aligned16(planes_r)) return MATQ_EALIGN;
+  const size_t need = packed_bytes(N, K, r);
+  if (bytes < need) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(cudaMemcpyAsync(planes_r, planes, need, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+}
+
+size_t matq_linear_workspace(int M, int K, int N, int group) {
+  (void)N;
+  if (M < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
+  return M <= kDecodeMaxM ? decode_workspace_bytes(M, K, group) : prefill_workspace_bytes(M, K, group);
+}
+
+int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
+                const uint8_t* zeros, int N, int r, int group, void* y, int y_mode, void* workspace,
+                size_t ws_bytes, void* stream) {
+  if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
+  if (r > r_keep) return MATQ_ETRUNC;
+  if (!valid_nk(N, K) || M < 1 || (long long)M * K > (1LL << 40) || (long long)M * N > (1LL << 40))
+    return MATQ_EINVAL_SHAPE;
+  if (group != 64 && group != 128) return MATQ_EINVAL_GROUP;
+  if (y_mode < MATQ_OUT_BF16 || y_mode > MATQ_OUT_F32_ACCUM) return MATQ_EDTYPE;
+  if (!x || !planes || !scales || !zeros || !y || !workspace) return MATQ_ENULL;
+  if (!aligned16(x) || !aligned16(planes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||
+      !aligned16(workspace))
+    return MATQ_EALIGN;
+  if (ws_bytes < matq_linear_workspace(M, K, N, group)) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  const PlaneGeom g = make_geom(N, K);
+  cudaError_t e;
+  if (M <= kDecodeMaxM)
+    e = launch_decode(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
+  else
+    e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
+  return cuda_status(e);
+}
+
+int matq_rmsnorm(const float* h, int M, int D, float eps, void* n_out, void* stream) {
+  if (M < 1 || D < 1 || (long long)M * D > (1LL << 40)) return MATQ_EINVAL_SHAPE;
+  if (!h || !n_out) return MATQ_ENULL;
+  if (!aligned16(h) || !aligned16(n_out)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_rmsnorm(h, M, D, eps, n_out, (cudaStream_t)stream));
+}
+
+int matq_silu_mul(const void* gate, const void* up, int M, int F, void* a_out, void* stream) {
+  if (M < 1 || F < 1 || (long long)M * F > (1LL << 40)) return MATQ_EINVAL_SHAPE;
+  if (!gate || !up || !a_out) return MATQ_ENULL;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(a_out)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_silu_mul(gate, up, M, F, a_out, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,70 @@
+// Glue of the Mix'n'Match FFN stack ("Matryoshka Quantization | Summary" §4.3, MatGPTQ §5.4):
+// unit-gain RMSNorm in front of the gate/up projections and the SiLU-gated product between
+// the two FFN halves.  The pages give no block formula; the reading taken is the Llama-style
+// block h <- h + down(silu(gate(n)) * up(n)), n = h / sqrt(mean(h^2) + eps).  Both kernels
+// are HBM-bound elementwise passes with fp32 arithmetic and bf16 outputs.
+#include "common.cuh"
+#include "internal.h"
+
+namespace matq {
+
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ h, int D, float eps,
+                                                      __nv_bfloat16* __restrict__ out) {
+  const int row = blockIdx.x;
+  const float* hr = h + (size_t)row * D;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) ss = fmaf(hr[i], hr[i], ss);
+  __shared__ float part[8];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
+  const float inv = rsqrtf(tot / (float)D + eps);
+  __nv_bfloat16* orow = out + (size_t)row * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) orow[i] = __float2bfloat16_rn(hr[i] * inv);
+}
+
+__device__ __forceinline__ float silu_f(float t) { return t / (1.0f + expf(-t)); }
+
+__global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __restrict__ gate,
+                                                       const __nv_bfloat16* __restrict__ up, size_t n,
+                                                       __nv_bfloat16* __restrict__ out) {
+  const size_t nvec = n / 8;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
+    const uint4 g4 = reinterpret_cast<const uint4*>(gate)[v];
+    const uint4 u4 = reinterpret_cast<const uint4*>(up)[v];
+    const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&g4);
+    const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&u4);
+    uint4 o4;
+    __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o4);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      ob[i] = __float2bfloat16_rn(silu_f(__bfloat162float(gb[i])) * __bfloat162float(ub[i]));
+    reinterpret_cast<uint4*>(out)[v] = o4;
+  }
+  // scalar tail
+  const size_t tail0 = nvec * 8;
+  for (size_t i = tail0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = __float2bfloat16_rn(silu_f(__bfloat162float(gate[i])) * __bfloat162float(up[i]));
+}
+
+cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s) {
+  rmsnorm_kernel<<<M, 256, 0, s>>>(h, D, eps, (__nv_bfloat16*)out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s) {
+  const size_t n = (size_t)M * F;
+  const size_t nvec = (n + 7) / 8;
+  int blocks = (int)((nvec + 255) / 256);
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  silu_mul_kernel<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)gate, (const __nv_bfloat16*)up, n,
+                                         (__nv_bfloat16*)out);
+  return cudaGetLastError();
+}
+
+}  // namespace matq

@@ -1,0 +1,28 @@
+// Launchers shared between libmatq's translation units (not part of the public ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include "common.cuh"
+
+namespace matq {
+
+cudaError_t launch_pack(const uint8_t* codes, const PlaneGeom& g, int r_keep, void* planes, cudaStream_t s);
+cudaError_t launch_slice(const void* planes, const PlaneGeom& g, int r, uint8_t* out, cudaStream_t s);
+
+size_t decode_workspace_bytes(int M, int K, int group);
+cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
+                          const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
+                          int y_mode, void* workspace, cudaStream_t s);
+
+size_t prefill_workspace_bytes(int M, int K, int group);
+cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
+                           const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
+                           int y_mode, void* workspace, cudaStream_t s);
+
+cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s);
+cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s);
+
+// Largest M served by the decode (mma.sync streaming) path; larger M takes the prefill path.
+constexpr int kDecodeMaxM = 16;
+
+}  // namespace matq

@@ -1,0 +1,170 @@
+"""ctypes binding of libmatq (C ABI declared in include/matq.h).
+
+Argument marshalling only: every step of the sliced linear layer runs in libmatq's CUDA
+kernels.  The functions named like the C entry points take raw pointers (ints) and sizes;
+the helpers below them take torch tensors (used for device memory and streams only) and
+raise ``MatqError`` on a non-zero status.  There is no CPU fallback: importing this module
+fails loudly when the shared library is missing.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmatq.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libmatq.so not found at {LIB_PATH}; build it with "
+        "`python -m nested_bit_weight_msb_b200.build` (needs nvcc)"
+    )
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status codes and output modes (mirror include/matq.h)
+MATQ_OK = 0
+MATQ_EINVAL_R = -1
+MATQ_EINVAL_SHAPE = -2
+MATQ_EINVAL_GROUP = -3
+MATQ_EALIGN = -4
+MATQ_ENULL = -5
+MATQ_ETRUNC = -6
+MATQ_ECUDA = -7
+MATQ_ESIZE = -8
+MATQ_EDTYPE = -9
+MATQ_EDEVICE = -10
+MATQ_OUT_BF16 = 0
+MATQ_OUT_F32 = 1
+MATQ_OUT_F32_ACCUM = 2
+
+WIDTHS = (2, 3, 4, 6, 8)
+DECODE_MAX_M = 16
+
+_c_int, _c_size, _c_vp, _c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+
+_SIGNATURES = {
+    "matq_version": (_c_int, []),
+    "matq_strerror": (ctypes.c_char_p, [_c_int]),
+    "matq_last_cuda_error": (_c_int, []),
+    "matq_plane_count": (_c_int, [_c_int]),
+    "matq_packed_bytes": (_c_size, [_c_int, _c_int, _c_int]),
+    "matq_pack": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_vp, _c_size, _c_vp]),
+    "matq_slice": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_int, _c_vp, _c_vp]),
+    "matq_slice_copy": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_int, _c_vp, _c_size, _c_vp]),
+    "matq_linear_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "matq_linear": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                             _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
+    "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
+    "matq_silu_mul": (_c_int, [_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_vp]),
+}
+
+for _name, (_res, _args) in _SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+    globals()[_name] = _fn
+
+EXPORTED = tuple(_SIGNATURES)
+
+
+class MatqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = matq_strerror(status).decode()
+        if status == MATQ_ECUDA:
+            msg += f" (cudaError {matq_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [status {status}]")
+
+
+def check(status: int, what: str) -> None:
+    if status != MATQ_OK:
+        raise MatqError(status, what)
+
+
+# ---------------------------------------------------------------------------------------
+# torch-tensor helpers (memory and streams only)
+# ---------------------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+def pack(codes, r_keep: int = 8, stream=None):
+    """Pack [N, K] uint8 codes (CUDA tensor) into a uint8 plane buffer (CUDA tensor)."""
+    torch = _torch()
+    N, K = codes.shape
+    nbytes = matq_packed_bytes(N, K, r_keep)
+    if nbytes == 0:
+        check(MATQ_EINVAL_SHAPE if r_keep in WIDTHS else MATQ_EINVAL_R, "matq_packed_bytes")
+    planes = torch.empty(nbytes, dtype=torch.uint8, device=codes.device)
+    check(matq_pack(_ptr(codes), N, K, r_keep, _ptr(planes), nbytes, _stream_ptr(stream)), "matq_pack")
+    return planes
+
+
+def slice_prefix(planes, N: int, K: int, r_keep: int, r: int, stream=None):
+    """Prefixes p = q >> (8 - r) as a [N, K] uint8 CUDA tensor."""
+    torch = _torch()
+    out = torch.empty((N, K), dtype=torch.uint8, device=planes.device)
+    check(matq_slice(_ptr(planes), N, K, r_keep, r, _ptr(out), _stream_ptr(stream)), "matq_slice")
+    return out
+
+
+def slice_copy(planes, N: int, K: int, r_keep: int, r: int, stream=None):
+    """Deployment mode A: a new plane buffer holding only the width-r prefix."""
+    torch = _torch()
+    nbytes = matq_packed_bytes(N, K, r)
+    out = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=planes.device)
+    check(matq_slice_copy(_ptr(planes), N, K, r_keep, r, _ptr(out), out.numel(), _stream_ptr(stream)),
+          "matq_slice_copy")
+    return out[:nbytes]
+
+
+def workspace_bytes(M: int, K: int, N: int, group: int) -> int:
+    return int(matq_linear_workspace(M, K, N, group))
+
+
+def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=None,
+           y_mode: int = MATQ_OUT_BF16, workspace=None, stream=None):
+    """y = x . W_hat_r^T.  x: [M, K] bf16 CUDA tensor; scales: [N, K/group] (fp16 or int16
+    bits); zeros: [N, K/group] uint8.  Returns y ([M, N] bf16 or fp32)."""
+    torch = _torch()
+    M, K = x.shape
+    if y is None:
+        dt = torch.bfloat16 if y_mode == MATQ_OUT_BF16 else torch.float32
+        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, N), dtype=dt, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
+    check(matq_linear(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
+                      _ptr(y), y_mode, _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "matq_linear")
+    return y
+
+
+def rmsnorm(h, eps: float = 1e-5, out=None, stream=None):
+    torch = _torch()
+    M, D = h.shape
+    if out is None:
+        out = torch.empty((M, D), dtype=torch.bfloat16, device=h.device)
+    check(matq_rmsnorm(_ptr(h), M, D, eps, _ptr(out), _stream_ptr(stream)), "matq_rmsnorm")
+    return out
+
+
+def silu_mul(gate, up, out=None, stream=None):
+    torch = _torch()
+    M, F = gate.shape
+    if out is None:
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=gate.device)
+    check(matq_silu_mul(_ptr(gate), _ptr(up), M, F, _ptr(out), _stream_ptr(stream)), "matq_silu_mul")
+    return out

@@ -1,0 +1,111 @@
+"""Host-side checks of the C-ABI library: it loads, exports every entry point the header
+declares, answers the layout queries, and rejects bad arguments with the documented
+status before touching a GPU (every call here fails validation, so none launches)."""
+
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "matq.h")
+
+
+@pytest.fixture(scope="module")
+def M():
+    from nested_bit_weight_msb_b200 import build
+    build.build()
+    from nested_bit_weight_msb_b200 import matq
+    return matq
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(matq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("matq_pack", "matq_slice", "matq_slice_copy", "matq_linear", "matq_linear_workspace",
+              "matq_packed_bytes", "matq_strerror"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(M):
+    import ctypes
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) == set(M.EXPORTED)
+
+
+def test_layout_queries(M):
+    assert [M.matq_plane_count(r) for r in (2, 3, 4, 6, 8)] == [1, 2, 3, 4, 5]
+    assert M.matq_plane_count(5) == 0 and M.matq_plane_count(1) == 0
+    for N, K in [(1024, 1024), (14336, 4096), (4096, 14336), (3584, 14336), (17, 256), (1, 512)]:
+        npad = (N + 15) // 16 * 16
+        for r in (2, 3, 4, 6, 8):
+            assert M.matq_packed_bytes(N, K, r) == npad * K * r // 8
+    # exactly r bits per weight on the benchmark shapes
+    assert M.matq_packed_bytes(14336, 4096, 2) == 14336 * 4096 * 2 // 8
+    assert M.matq_packed_bytes(1024, 1000, 4) == 0          # K not a multiple of 256
+    assert M.matq_packed_bytes(0, 1024, 4) == 0
+    assert M.matq_packed_bytes(16, 1024, 5) == 0
+    assert M.matq_version() >= 100
+    assert M.matq_strerror(M.MATQ_ETRUNC).decode().startswith("pack holds")
+
+
+def test_workspace_query(M):
+    assert M.matq_linear_workspace(1, 4096, 14336, 128) > 0
+    assert M.matq_linear_workspace(1, 4096, 14336, 128) % 256 == 0
+    assert M.matq_linear_workspace(2048, 4096, 14336, 128) >= 2048 * 4096 * 2
+    assert M.matq_linear_workspace(1, 4096, 14336, 96) == 0
+
+
+FAKE = 1 << 20          # non-null, 16-byte aligned, never dereferenced (validation fails first)
+
+
+def test_pack_rejects(M):
+    assert M.matq_pack(FAKE, 16, 1024, 5, FAKE, 1 << 30, None) == M.MATQ_EINVAL_R
+    assert M.matq_pack(FAKE, 16, 1000, 4, FAKE, 1 << 30, None) == M.MATQ_EINVAL_SHAPE
+    assert M.matq_pack(FAKE, 0, 1024, 4, FAKE, 1 << 30, None) == M.MATQ_EINVAL_SHAPE
+    assert M.matq_pack(None, 16, 1024, 4, FAKE, 1 << 30, None) == M.MATQ_ENULL
+    assert M.matq_pack(FAKE + 8, 16, 1024, 4, FAKE, 1 << 30, None) == M.MATQ_EALIGN
+    assert M.matq_pack(FAKE, 16, 1024, 4, FAKE, 16 * 1024 * 4 // 8 - 1, None) == M.MATQ_ESIZE
+
+
+def test_slice_rejects(M):
+    assert M.matq_slice(FAKE, 16, 1024, 4, 6, FAKE, None) == M.MATQ_ETRUNC
+    assert M.matq_slice(FAKE, 16, 1024, 4, 5, FAKE, None) == M.MATQ_EINVAL_R
+    assert M.matq_slice(FAKE, 16, 1024, 8, 4, None, None) == M.MATQ_ENULL
+    assert M.matq_slice_copy(FAKE, 16, 1024, 8, 4, FAKE, 16 * 1024 * 4 // 8 - 16, None) == M.MATQ_ESIZE
+    assert M.matq_slice_copy(FAKE, 16, 1024, 2, 4, FAKE, 1 << 20, None) == M.MATQ_ETRUNC
+
+
+def test_linear_rejects(M):
+    ws = 1 << 30
+
+    def call(**kw):
+        a = dict(x=FAKE, M=1, K=1024, planes=FAKE, r_keep=8, scales=FAKE, zeros=FAKE, N=64, r=4, group=128,
+                 y=FAKE, y_mode=0, ws=FAKE, ws_bytes=ws)
+        a.update(kw)
+        return M.matq_linear(a["x"], a["M"], a["K"], a["planes"], a["r_keep"], a["scales"], a["zeros"], a["N"],
+                             a["r"], a["group"], a["y"], a["y_mode"], a["ws"], a["ws_bytes"], None)
+
+    assert call(r=5) == M.MATQ_EINVAL_R
+    assert call(r=8, r_keep=4) == M.MATQ_ETRUNC
+    assert call(M=0) == M.MATQ_EINVAL_SHAPE
+    assert call(K=1000) == M.MATQ_EINVAL_SHAPE
+    assert call(N=0) == M.MATQ_EINVAL_SHAPE
+    assert call(group=32) == M.MATQ_EINVAL_GROUP
+    assert call(y_mode=3) == M.MATQ_EDTYPE
+    assert call(x=None) == M.MATQ_ENULL
+    assert call(zeros=FAKE + 4) == M.MATQ_EALIGN
+    assert call(ws_bytes=16) == M.MATQ_ESIZE
+
+
+def test_glue_rejects(M):
+    assert M.matq_rmsnorm(FAKE, 0, 16, 1e-5, FAKE, None) == M.MATQ_EINVAL_SHAPE
+    assert M.matq_rmsnorm(None, 1, 16, 1e-5, FAKE, None) == M.MATQ_ENULL
+    assert M.matq_silu_mul(FAKE, FAKE + 2, 1, 16, FAKE, None) == M.MATQ_EALIGN

@@ -1,0 +1,143 @@
+"""GPU parity of matq_linear against the fp64 oracle.
+
+Decode path (M <= 16) and prefill path (M > 16), all widths, both group sizes, every
+output mode; small shapes that span several tiles with ragged tails compared element by
+element; the benchmark shapes compared on sampled output rows (the oracle computes those
+rows one by one).  Bar: |y - ref| <= 1e-2 (|ref| + 1) elementwise and relative Frobenius
+error <= 2e-3 (tests/helpers.py).
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from helpers import check_close, problem, to_device
+from nested_bit_weight_msb_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from nested_bit_weight_msb_b200 import matq
+    return matq
+
+
+def run(M, q, s, z, xb, r, group, r_keep=8, y_mode=0):
+    import torch
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=r_keep)
+    y = M.linear(dx, planes, r_keep, ds, dz, q.shape[0], r, group, y_mode=y_mode)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy()
+
+
+# ---- decode path -------------------------------------------------------------------------
+
+@pytest.mark.parametrize("r", O.WIDTHS)
+def test_single_linear_1024(M, r):
+    """K = N = 1024, group 128, M = 1, seed 0 (the single-linear-layer workload)."""
+    q, s, z, xb, xv = problem(1, 1024, 1024, 128, seed=0)
+    ref = O.linear(xv, q, s, z, r, 128)
+    for mode in (M.MATQ_OUT_BF16, M.MATQ_OUT_F32):
+        y = run(M, q, s, z, xb, r, 128, y_mode=mode)
+        check_close(y, ref, what=f"r={r} mode={mode}")
+
+
+@pytest.mark.parametrize("group", [64, 128])
+@pytest.mark.parametrize("Mt", [1, 2, 3, 5, 8, 9, 12, 16])
+def test_decode_small_sweep(M, Mt, group):
+    """Several row tiles with a ragged last tile, several chunks, every width."""
+    N, K = 83, 768
+    q, s, z, xb, xv = problem(Mt, N, K, group, seed=Mt + group)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    for r in O.WIDTHS:
+        ref = O.linear(xv, q, s, z, r, group)
+        y = M.linear(dx, planes, 8, ds, dz, N, r, group, y_mode=M.MATQ_OUT_F32).cpu().numpy()
+        check_close(y, ref, what=f"M={Mt} g={group} r={r}")
+
+
+def test_decode_accumulate_mode(M):
+    import torch
+    N, K, Mt = 130, 512, 4
+    q, s, z, xb, xv = problem(Mt, N, K, 64, seed=5)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    base = np.random.default_rng(1).standard_normal((Mt, N)).astype(np.float32)
+    y = torch.from_numpy(base.copy()).cuda()
+    M.linear(dx, planes, 8, ds, dz, N, 3, 64, y=y, y_mode=M.MATQ_OUT_F32_ACCUM)
+    check_close(y.cpu().numpy(), base + O.linear(xv, q, s, z, 3, 64), what="accumulate")
+
+
+@pytest.mark.parametrize("r", O.WIDTHS)
+def test_truncated_pack_gives_identical_output(M, r):
+    """Mode A (only the r-bit prefix resident) and mode B (all 8 bits, r per call) read the
+    same bits, so the outputs are bitwise equal."""
+    import torch
+    N, K, Mt = 64, 1024, 3
+    q, s, z, xb, xv = problem(Mt, N, K, 128, seed=r)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    full = M.pack(dq, r_keep=8)
+    trunc = M.slice_copy(full, N, K, 8, r)
+    a = M.linear(dx, full, 8, ds, dz, N, r, 128, y_mode=M.MATQ_OUT_F32)
+    b = M.linear(dx, trunc, r, ds, dz, N, r, 128, y_mode=M.MATQ_OUT_F32)
+    assert torch.equal(a, b)
+
+
+def test_decode_closed_forms(M):
+    import torch
+    N, K = 32, 512
+    # codes equal to their zero point at r = 8: W_hat = 0, so y = 0
+    rng = np.random.default_rng(3)
+    z = rng.integers(0, 256, (N, K // 128), dtype=np.uint8)
+    q = np.repeat(z, 128, axis=1)
+    s = rng.uniform(1e-3, 1e-2, (N, K // 128)).astype(np.float16)
+    xb, xv = synth.bf16_round(rng.standard_normal((2, K)).astype(np.float32))
+    y = run(M, q, s, z, xb, 8, 128, y_mode=M.MATQ_OUT_F32)
+    # the exact result is 0; fp32 rounding of the cancelling terms s*z*sum(x) stays tiny
+    scale = float((s.astype(np.float64) * z).max()) * float(np.abs(xv).sum())
+    assert np.max(np.abs(y)) <= 1e-5 * scale
+    # one-hot activations pick a column of W_hat
+    q = rng.integers(0, 256, (N, K), dtype=np.uint8)
+    for k in (0, 7, 8, 15, 200, 511):
+        e = np.zeros((1, K), dtype=np.float32)
+        e[0, k] = 1.0
+        eb, ev = synth.bf16_round(e)
+        for r in O.WIDTHS:
+            y = run(M, q, s, z, eb, r, 128, y_mode=M.MATQ_OUT_F32)
+            col = O.dequant(q, s, z, r, 128)[:, k]
+            assert np.allclose(y[0], col, rtol=1e-5, atol=1e-6), (k, r)
+
+
+def test_decode_outlier_activations(M):
+    N, K = 256, 4096
+    q, s, z, xb, xv = problem(16, N, K, 128, seed=9, outlier_frac=0.01)
+    for r in O.WIDTHS:
+        check_close(run(M, q, s, z, xb, r, 128), O.linear(xv, q, s, z, r, 128), what=f"r={r}")
+
+
+@pytest.mark.parametrize("shape,group", [((14336, 4096), 128), ((4096, 14336), 128),
+                                         ((14336, 3584), 64), ((3584, 14336), 64)])
+def test_decode_full_size_sampled(M, shape, group):
+    """Benchmark FFN shapes (8B gate/up and down, g=128; 9B gate/up and down, g=64) at the
+    decode batch sizes, every width, in the same launch configuration the bench times;
+    64 sampled output rows are checked against the oracle."""
+    import torch
+    N, K = shape
+    q, s, z = synth.parent_weights(N, K, group, seed=0, proj="gate" if N > K else "down")
+    dq = torch.from_numpy(q).cuda()
+    ds = torch.from_numpy(s.view(np.int16)).cuda()
+    dz = torch.from_numpy(z).cuda()
+    planes = M.pack(dq, r_keep=8)
+    rows = np.sort(np.random.default_rng(N).choice(N, 64, replace=False))
+    for Mt in (1, 4, 16):
+        xb, xv = synth.activations(Mt, K, seed=0)
+        dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        for r in O.WIDTHS:
+            y = M.linear(dx, planes, 8, ds, dz, N, r, group).float().cpu().numpy()
+            ref = O.linear(xv, q[rows], s[rows], z[rows], r, group)
+            check_close(y[:, rows], ref, what=f"{shape} M={Mt} r={r}")
