@@ -1,0 +1,452 @@
+"""Benchmark of the sliced r-bit linear layer (MatQuant / MatGPTQ true-prefix slicing) on B200.
+
+Workload (default, ``--workload ffn8b_decode``): the Llama-3.1-8B-shaped FFN at decode
+batch sizes.  One step runs, for every width r in {2, 3, 4, 6, 8} and every batch
+M in {1, 4, 16}, one FFN forward through the sliced linears:
+    gate = x . W_gate,r^T   [M, 14336]      (matq_linear, decode path)
+    up   = x . W_up,r^T     [M, 14336]
+    a    = silu(gate) * up                  (matq_silu_mul)
+    y    = a . W_down,r^T   [M, 4096]
+with group-128 parent codes of N(0, 0.02) weights (synthetic, seeded) and N(0, 1) bf16
+activations.  ``value`` = algorithmic bytes of the sliced linears (planes of width r,
+fp16 scales, uint8 zeros, x, y) over the device time of the step -> GB/s.
+
+``--workload ffn8b_prefill``: the same FFN at M = 2048 with 1% outlier channels x20,
+r in {3, 4, 8}; ``value`` = 2*M*N*K flops of the sliced linears over the step time -> TFLOP/s.
+
+L2 (126 MB) is defeated by rotating through several device copies of the packed layer
+(working set > 1 GB), so every call streams its planes from HBM.
+
+Multi-GPU (torchrun, one rank per GPU): replicas / weak scaling -- every rank serves its own
+batches with its own copy of the weights; there is no exchange step on this path.  The
+step time is the max over ranks (device events, all-reduced).
+
+``--impl reference``: the fp64 CPU oracle (the only reference this method has here), timed
+on a bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+
+WIDTHS = (2, 3, 4, 6, 8)
+D_MODEL, D_FF, GROUP = 4096, 14336, 128
+METRIC = "sliced r-bit linear: decode weight GB/s vs HBM peak; prefill TFLOP/s per r"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
+    ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_spec(name):
+    if name == "ffn8b_decode":
+        return dict(widths=WIDTHS, batches=(1, 4, 16), outlier=0.0, unit="GB/s")
+    return dict(widths=(3, 4, 8), batches=(2048,), outlier=0.01, unit="TFLOP/s")
+
+
+def linear_bytes(M, N, K, r, group=GROUP):
+    G = K // group
+    return N * K * r // 8 + N * G * 3 + M * K * 2 + M * N * 2
+
+
+def step_units(spec):
+    """(algorithmic bytes, flops) of one step."""
+    b = f = 0
+    for r in spec["widths"]:
+        for M in spec["batches"]:
+            for (N, K) in ((D_FF, D_MODEL), (D_FF, D_MODEL), (D_MODEL, D_FF)):
+                b += linear_bytes(M, N, K, r)
+                f += 2 * M * N * K
+    return b, f
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def maybe_init_pg(world, backend):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value, device):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------------------------
+
+def cpu_oracle_rate(spec, weights_host, budget_s=12.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: rows of
+    the three FFN matrices at each (r, M), scaled to the metric's unit per second."""
+    import oracle as O
+    rows = 256
+    done_b = done_f = 0.0
+    t0 = time.perf_counter()
+    rng = np.random.default_rng(0)
+    n_iter = 0
+    while time.perf_counter() - t0 < budget_s or n_iter == 0:
+        for r in spec["widths"]:
+            for M in spec["batches"]:
+                for name, (N, K) in (("gate", (D_FF, D_MODEL)), ("up", (D_FF, D_MODEL)), ("down", (D_MODEL, D_FF))):
+                    q, s, z = weights_host[name]
+                    Mi = min(M, 64)
+                    x = rng.standard_normal((Mi, K))
+                    O.linear(x, q[:rows], s[:rows], z[:rows], r, GROUP)
+                    done_b += linear_bytes(Mi, rows, K, r)
+                    done_f += 2 * Mi * rows * K
+        n_iter += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=cores)
+    except Exception:
+        pass
+    val = done_b / dt / 1e9 if spec["unit"] == "GB/s" else done_f / dt / 1e12
+    sample = (f"first {rows} rows of gate/up/down at every (r, M) of the workload "
+              f"(M capped at 64), {n_iter} pass(es), {dt:.1f} s")
+    return {"value": val, "unit": spec["unit"], "cores": cores, "kind": "oracle", "sample": sample}
+
+
+def host_weights():
+    from nested_bit_weight_msb_b200 import synth
+    return {name: synth.parent_weights(N, K, GROUP, seed=0, layer=0, proj=name)
+            for name, (N, K) in (("gate", (D_FF, D_MODEL)), ("up", (D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))}
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the oracle on the host
+# ---------------------------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, local = dist_setup()
+    if rank != 0:
+        return 0
+    spec = workload_spec(args.workload)
+    w = host_weights()
+    for _ in range(args.warmup):
+        cpu_oracle_rate(spec, w, budget_s=0.5)
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_oracle_rate(spec, w, budget_s=5.0))
+    v = float(np.mean([c["value"] for c in vals]))
+    b, f = step_units(spec)
+    per_step_units = b / 1e9 if spec["unit"] == "GB/s" else f / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": spec["unit"], "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_units / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "device": "cpu"},
+        "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"], "value": v,
+                         "unit": spec["unit"]},
+        "e2e": {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    maybe_init_pg(world, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from nested_bit_weight_msb_b200 import matq, synth
+
+    spec = workload_spec(args.workload)
+    weights = host_weights()
+    # pack once per matrix (one-time), then clone into rotating copies
+    packed = {}
+    meta = {}
+    for name, (q, s, z) in weights.items():
+        dq = torch.from_numpy(q).to(dev)
+        p = matq.pack(dq, r_keep=8)
+        packed[name] = [p] + [p.clone() for _ in range(args.copies - 1)]
+        meta[name] = (torch.from_numpy(s.view(np.int16)).to(dev), torch.from_numpy(z).to(dev), q.shape[0], q.shape[1])
+        del dq
+    torch.cuda.synchronize()
+
+    batches = spec["batches"]
+    xs = {}
+    for M in batches:
+        xb, _ = synth.activations(M, D_MODEL, seed=rank, outlier_frac=spec["outlier"])
+        xs[M] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    Mmax = max(batches)
+    ws = torch.empty(max(matq.workspace_bytes(Mmax, D_FF, D_FF, GROUP), matq.workspace_bytes(Mmax, D_MODEL, D_FF, GROUP)),
+                     dtype=torch.uint8, device=dev)
+    gate_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
+    up_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
+    a_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
+    y_buf = {M: torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev) for M in batches}
+
+    def linear(name, copy, x, r, out):
+        s, z, N, K = meta[name]
+        matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, workspace=ws)
+
+    def ffn(x, M, r, copy):
+        linear("gate", copy, x, r, gate_buf[M])
+        linear("up", copy, x, r, up_buf[M])
+        matq.silu_mul(gate_buf[M], up_buf[M], out=a_buf[M])
+        linear("down", copy, a_buf[M], r, y_buf[M])
+
+    calls = [(r, M) for r in spec["widths"] for M in batches]
+
+    def step(base=0):
+        for i, (r, M) in enumerate(calls):
+            ffn(xs[M], M, r, (base + i) % args.copies)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local) as clk:
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+    ms_total = max_over_ranks(world, e0.elapsed_time(e1), dev)
+    ms_step = ms_total / args.steps
+    b, f = step_units(spec)
+    if spec["unit"] == "GB/s":
+        value = b * world / (ms_step * 1e-3) / 1e9
+    else:
+        value = f * world / (ms_step * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel: per-call device time of the sliced linear ----------
+    rl = roofline(args, spec, linear, xs, gate_buf, stream, dev)
+
+    # ---- end-to-end through the public API with host buffers --------------------------------
+    e2e = end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world)
+
+    line = None
+    if rank == 0:
+        peaks = load_peaks()
+        line = {
+            "metric": METRIC, "value": value, "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16-operands/f32-acc (bf16 in/out)", "data": "synthetic",
+            "config": {"workload": args.workload, "shapes": "gate/up [14336,4096], down [4096,14336], group 128",
+                       "widths": list(spec["widths"]), "batches": list(batches),
+                       "l2": f"rotating {args.copies} device copies of the packed layer (> L2)",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graph replay, CUDA events"},
+            "roofline": rl,
+            "e2e": e2e,
+            "gpu_launches": args.steps * len(calls) * (3 * 2 + 1),
+            "clocks": clk.summary(),
+            "peaks_source": peaks.get("_source"),
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_rate(spec, weights)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graph
+        dist.destroy_process_group()
+    return 0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        d["_source"] = "measured"
+        return d
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_source": "fallback"}
+
+
+def roofline(args, spec, linear, xs, gate_buf, stream, dev):
+    """Average device duration of single sliced-linear calls (the dominant kernel and its
+    activation pre-pass), measured with CUDA events on the launching stream while a
+    preceding spin kernel keeps the host ahead of the device."""
+    import torch
+    peaks = load_peaks()
+    M = max(spec["batches"]) if spec["unit"] == "TFLOP/s" else 1
+    r = 2 if spec["unit"] == "GB/s" else 4
+    n = 24
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(2e8))
+        for i in range(n):
+            ev[i].record(stream)
+            linear("gate", i % args.copies, xs[M], r, gate_buf[M])
+        ev[n].record(stream)
+        torch.cuda.synchronize()
+    durs = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+    avg_ms = float(np.mean(durs[2:]))
+    if spec["unit"] == "GB/s":
+        units = linear_bytes(M, D_FF, D_MODEL, r)
+        ach = units / (avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": None, "kernel": f"matq_linear decode (gate 14336x4096, r={r}, M={M}), per call",
+                "avg_us": avg_ms * 1e3, "peak_source": peaks.get("_source")}
+    flops = 2 * M * D_FF * D_MODEL
+    ach = flops / (avg_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+            "traffic": None, "kernel": f"matq_linear prefill (gate 14336x4096, r={r}, M={M}), per call",
+            "avg_us": avg_ms * 1e3, "peak_source": peaks.get("_source")}
+
+
+def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
+    """The same step through the public calls, with each call's activations copied in from
+    pinned host memory and its output copied back, inside the timed region."""
+    import torch
+    host_x = {M: xs[M].cpu().pin_memory() for M in xs}
+    host_y = {M: torch.empty_like(y_buf[M], device="cpu").pin_memory() for M in y_buf}
+    dev_x = {M: torch.empty_like(xs[M]) for M in xs}
+    h2d = sum(host_x[M].numel() * 2 for (_, M) in calls)
+    d2h = sum(host_y[M].numel() * 2 for (_, M) in calls)
+
+    def step(base=0):
+        for i, (r, M) in enumerate(calls):
+            dev_x[M].copy_(host_x[M], non_blocking=True)
+            ffn(dev_x[M], M, r, (base + i) % args.copies)
+            host_y[M].copy_(y_buf[M], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(world, e0.elapsed_time(e1), dev) / args.steps
+    b, f = step_units(spec)
+    v = (b * world / (ms * 1e-3) / 1e9) if spec["unit"] == "GB/s" else (f * world / (ms * 1e-3) / 1e12)
+    return {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,17 +1,540 @@
-// Prefill path (M > 16): placeholder until the tcgen05 kernel lands.
+// Prefill path (M > 16): TMA + tcgen05 GEMM over the packed r-bit planes.
+//
+// y = x . W_hat_r^T with W_hat = s * (q_hat - z), q_hat = p * 2^(8-r) + delta_r ("MatGPTQ:
+// Efficient and Accurate Inference over Nested Quantized Models", App. A.1 and §4).  This
+// path is a dense contraction, so it runs on the 5th-generation tensor cores:
+//
+//   * warp 0 (one thread) streams, with TMA, the raw planes of width r for a 128-row x
+//     256-input block (only those planes: exactly r bits per weight cross HBM) and the fp16
+//     activation tiles [BN tokens x 64 inputs] (128-byte swizzle, the UMMA K-major layout);
+//   * warps 4..7 turn each 64-input slice of the raw planes into an fp16 weight tile
+//     [128 x 64] in shared memory: operand registers are built from the plane words exactly
+//     as on the decode path (1024 + sigma*v), the exact code difference q_hat - z is formed
+//     in fp16 (exact: a half-integer below 256 in magnitude), and one fp16 multiply by the
+//     scale gives W_hat with a single rounding.  stmatrix writes the tiles in the swizzled
+//     layout; fence.proxy.async hands them to the tensor core;
+//   * warp 1 (one thread) issues tcgen05.mma (M = 128 weight rows, N = BN tokens, K = 16)
+//     accumulating in TMEM, and releases ring slots with tcgen05.commit;
+//   * warps 4..7 then read the fp32 accumulator with tcgen05.ld and store y.
+//
+// fp16 (not bf16) weight tiles: with bf16 y, bf16-rounded weights exceed the 2e-3 relative
+// error budget while fp16 ones stay at the output-rounding level; both formats run at the
+// same tensor-core rate.  x is converted bf16 -> fp16 once per call into the workspace (exact
+// for |x| in the fp16 normal range).
+//
+// Every mbarrier wait is bounded (about a second of clock); on expiry the kernel records an
+// error code in the workspace flag, every role drains, TMEM is freed, and the kernel returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "operands.cuh"
 
 namespace matq {
 
-size_t prefill_workspace_bytes(int M, int K, int group) {
-  (void)group;
-  return (((size_t)M * K * 2) + 255) & ~size_t(255);
+constexpr int kBM = 128;        // weight rows per tile (UMMA M)
+constexpr int kSubK = 64;       // inputs per A/B ring slot (one 128-byte swizzle row of fp16)
+constexpr int kRawStages = 2;   // raw-plane ring (256 inputs per slot)
+constexpr int kAStages = 3;     // fp16 weight-tile ring
+constexpr int kBStages = 3;     // activation-tile ring
+constexpr int kThreads = 256;
+constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
+constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+
+// ---- PTX wrappers --------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false (and the error flag set) if the phase did not complete in time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(err, code);
+      return false;
+    }
+  }
+  return true;
 }
 
-cudaError_t launch_prefill(const void*, int, int, const void*, const PlaneGeom&, const uint16_t*, const uint8_t*, int,
-                           int, void*, int, void*, cudaStream_t) {
-  return cudaErrorNotSupported;
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// SW128 K-major shared-memory matrix descriptor (rows of 128 bytes, 8-row groups 1024 B apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void stmatrix_x4(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- activation conversion -----------------------------------------------------------------
+__global__ void xprep_prefill_kernel(const uint16_t* __restrict__ x, size_t n, __half* __restrict__ x16,
+                                     int* __restrict__ err) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
+  const size_t nvec = n / 8;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
+    const uint4 in = reinterpret_cast<const uint4*>(x)[v];
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint4 out;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
+      __half2 h = __floats2half2_rn(a, b);
+      o[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(x16)[v] = out;
+  }
+}
+
+// ---- the GEMM kernel -----------------------------------------------------------------------
+struct PrefillParams {
+  int M, N, K, G, RT;
+  const uint16_t* scales;
+  const uint8_t* zeros;
+  void* y;
+  int y_mode;
+  int* err;
+};
+
+template <int R>
+__host__ __device__ constexpr int raw_stage_bytes() { return 4096 * R; }  // 8 row tiles x r bits x 512 B
+
+template <int R, int BN>
+struct PrefillSmem {
+  static constexpr int kA = 0;
+  static constexpr int kB = kA + kAStages * kATileBytes;
+  static constexpr int kRaw = kB + kBStages * BN * 128;
+  static constexpr int kBar = kRaw + kRawStages * raw_stage_bytes<R>();
+  static constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 1;
+  static constexpr int kTmemSlot = kBar + 8 * kNumBars;
+  static constexpr int kTotal = kTmemSlot + 16 + 1024;  // + alignment slack
+};
+
+// Byte offset of plane p inside a raw stage: planes are stored back to back, 8 row tiles each.
+__device__ __forceinline__ int raw_plane_off(int p) {
+  return p == 0 ? 0 : p == 1 ? 8192 : p == 2 ? 12288 : p == 3 ? 16384 : 24576;
+}
+
+// Read one lane's plane words of one row tile from a raw stage in shared memory.
+template <int R>
+__device__ __forceinline__ void lds_lane_words(const uint8_t* raw, int t, int lane, LaneWords& L) {
+  {
+    const uint8_t* b = raw + raw_plane_off(0) + t * 1024 + lane * 16;
+    const uint4 a = *reinterpret_cast<const uint4*>(b), c = *reinterpret_cast<const uint4*>(b + 512);
+    L.p0[0] = a.x; L.p0[1] = a.y; L.p0[2] = a.z; L.p0[3] = a.w;
+    L.p0[4] = c.x; L.p0[5] = c.y; L.p0[6] = c.z; L.p0[7] = c.w;
+  }
+  if constexpr (R >= 3) {
+    const uint4 a = *reinterpret_cast<const uint4*>(raw + raw_plane_off(1) + t * 512 + lane * 16);
+    L.p1[0] = a.x; L.p1[1] = a.y; L.p1[2] = a.z; L.p1[3] = a.w;
+  }
+  if constexpr (R >= 4) {
+    const uint4 a = *reinterpret_cast<const uint4*>(raw + raw_plane_off(2) + t * 512 + lane * 16);
+    L.p2[0] = a.x; L.p2[1] = a.y; L.p2[2] = a.z; L.p2[3] = a.w;
+  }
+  if constexpr (R >= 6) {
+    const uint8_t* b = raw + raw_plane_off(3) + t * 1024 + lane * 16;
+    const uint4 a = *reinterpret_cast<const uint4*>(b), c = *reinterpret_cast<const uint4*>(b + 512);
+    L.p3[0] = a.x; L.p3[1] = a.y; L.p3[2] = a.z; L.p3[3] = a.w;
+    L.p3[4] = c.x; L.p3[5] = c.y; L.p3[6] = c.z; L.p3[7] = c.w;
+  }
+  if constexpr (R >= 8) {
+    const uint8_t* b = raw + raw_plane_off(4) + t * 1024 + lane * 16;
+    const uint4 a = *reinterpret_cast<const uint4*>(b), c = *reinterpret_cast<const uint4*>(b + 512);
+    L.p4[0] = a.x; L.p4[1] = a.y; L.p4[2] = a.z; L.p4[3] = a.w;
+    L.p4[4] = c.x; L.p4[5] = c.y; L.p4[6] = c.z; L.p4[7] = c.w;
+  }
+}
+
+// Multiplier m_rho = 2^(8-r) / sigma_rho turning (A - 1024) into 2^(8-r) * p.
+template <int R>
+__device__ __forceinline__ float code_mult(int rho) {
+  if constexpr (R == 2) return (float)(64 >> (2 * rho));
+  else if constexpr (R == 3) return rho < 2 ? 32.f : 2.f;
+  else if constexpr (R == 4) return rho < 2 ? 16.f : 1.f;
+  else return 1.f;
+}
+
+// Dequantise the two MMA tiles of block W for one row tile and store them into the A slot.
+// rows: sr[0] / dz[0] for row gid, sr[1] / dz[1] for row gid + 8 (fp16 pairs, both halves equal).
+template <int R, int W>
+__device__ __forceinline__ void dequant_block(const LaneWords& L, const __half2 (&s2)[2], const __half2 (&dz2)[2],
+                                              uint32_t a_slot, int t, int lane) {
+  uint32_t A[2][4];
+  build_operands<R, W>(L, A);
+  const __half2 k1024 = __float2half2_rn(1024.f);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    uint32_t o[4];
+#pragma unroll
+    for (int rho = 0; rho < 4; ++rho) {
+      const __half2 v = *reinterpret_cast<const __half2*>(&A[j][rho]);
+      const int rsel = rho & 1;  // rho 0, 2: row gid; rho 1, 3: row gid + 8
+      __half2 u;
+      if constexpr (R == 8) {
+        u = __hsub2(v, __hadd2(k1024, dz2[rsel]));  // dz2 holds -z here: v - 1024 - z, exact
+      } else {
+        u = __hfma2(__hsub2(v, k1024), __float2half2_rn(code_mult<R>(rho)), dz2[rsel]);
+      }
+      const __half2 w = __hmul2(u, s2[rsel]);
+      o[rho] = *reinterpret_cast<const uint32_t*>(&w);
+    }
+    // stmatrix: lane i addresses row (i % 8) of matrix (i / 8); matrices 0..3 = (rows 0-7,
+    // k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15) of this 16x16 tile.
+    const int mi = lane >> 3;
+    const int row = t * 16 + (lane & 7) + 8 * (mi & 1);
+    const int kloc = 32 * (W & 1) + 16 * j + 8 * (mi >> 1);  // input within the 64-wide slot
+    const int chunk16 = kloc >> 3;
+    const uint32_t addr = a_slot + row * 128 + ((chunk16 ^ (row & 7)) << 4);
+    stmatrix_x4(addr, o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int R, int BN, int GROUP, int Q>
+__device__ __forceinline__ void dequant_substage(const LaneWords (&L)[2], const PrefillParams& P, int kc, int rt0,
+                                                 int wq, int lane, uint32_t a_slot) {
+  const int gid = lane >> 2;
+  const int gi = (kc * kChunk + Q * kSubK) / GROUP;
+  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt) {
+    const int t = 2 * wq + tt;
+    __half2 s2[2], dz2[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = (rt0 + t) * kTileRows + gid + 8 * h;
+      float s = 0.f, zf = 0.f;
+      if (row < P.N) {
+        s = __half2float(__ushort_as_half(P.scales[(size_t)row * P.G + gi]));
+        zf = (float)P.zeros[(size_t)row * P.G + gi];
+      }
+      s2[h] = __float2half2_rn(s);
+      dz2[h] = __float2half2_rn(R == 8 ? zf : (kDelta - zf));
+    }
+    dequant_block<R, 2 * Q>(L[tt], s2, dz2, a_slot, t, lane);
+    dequant_block<R, 2 * Q + 1>(L[tt], s2, dz2, a_slot, t, lane);
+  }
+}
+
+template <int R, int BN, int GROUP>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant__ CUtensorMap tm_p1,
+               const __grid_constant__ CUtensorMap tm_p2, const __grid_constant__ CUtensorMap tm_p3,
+               const __grid_constant__ CUtensorMap tm_p4, const __grid_constant__ CUtensorMap tm_x,
+               const PrefillParams P) {
+  using S = PrefillSmem<R, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* raw_full = bars;
+  uint64_t* raw_empty = raw_full + kRawStages;
+  uint64_t* a_full = raw_empty + kRawStages;
+  uint64_t* a_empty = a_full + kAStages;
+  uint64_t* b_full = a_empty + kAStages;
+  uint64_t* b_empty = b_full + kBStages;
+  uint64_t* acc_full = b_empty + kBStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rt0 = blockIdx.x * (kBM / kTileRows);
+  const int n0 = blockIdx.x * kBM;
+  const int m0 = blockIdx.y * BN;
+  const int KC = P.K / kChunk;
+  constexpr int kNumPlanes = planes_for_width(R);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRawStages; ++i) { mbar_init(&raw_full[i], 1); mbar_init(&raw_empty[i], 4); }
+    for (int i = 0; i < kAStages; ++i) { mbar_init(&a_full[i], 128); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < kBStages; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
+    mbar_init(acc_full, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const CUtensorMap* maps[5] = {&tm_p0, &tm_p1, &tm_p2, &tm_p3, &tm_p4};
+      bool ok = true;
+      for (int kc = 0; kc < KC && ok; ++kc) {
+        const int rs = kc % kRawStages;
+        ok = mbar_wait(&raw_empty[rs], ((kc / kRawStages) & 1) ^ 1, P.err, 1);
+        if (!ok) break;
+        mbar_expect_tx(&raw_full[rs], raw_stage_bytes<R>());
+        uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
+#pragma unroll
+        for (int p = 0; p < kNumPlanes; ++p)
+          tma_load_2d(raw + raw_plane_off(p), maps[p], kc * plane_bits(p) * 64, rt0, &raw_full[rs]);
+        for (int q = 0; q < 4; ++q) {
+          const int i = kc * 4 + q, bs = i % kBStages;
+          ok = mbar_wait(&b_empty[bs], ((i / kBStages) & 1) ^ 1, P.err, 2);
+          if (!ok) break;
+          mbar_expect_tx(&b_full[bs], BN * 128);
+          tma_load_2d(smem + S::kB + bs * BN * 128, &tm_x, kc * kChunk + q * kSubK, m0, &b_full[bs]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+      bool ok = true;
+      const int nsub = KC * 4;
+      for (int i = 0; i < nsub && ok; ++i) {
+        const int as = i % kAStages, bs = i % kBStages;
+        ok = mbar_wait(&a_full[as], (i / kAStages) & 1, P.err, 4) && mbar_wait(&b_full[bs], (i / kBStages) & 1, P.err, 8);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + S::kA + as * kATileBytes);
+        const uint32_t b_base = smem_u32(smem + S::kB + bs * BN * 128);
+#pragma unroll
+        for (int kk = 0; kk < kSubK / 16; ++kk)
+          tc_mma_f16(tmem_d, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&a_empty[as]);
+        tc_commit(&b_empty[bs]);
+      }
+      if (ok) tc_commit(acc_full);
+    }
+  } else if (warp >= 4) {
+    // ---------------- dequantisation, then epilogue ----------------
+    const int wq = warp - 4;
+    bool ok = true;
+    for (int kc = 0; kc < KC && ok; ++kc) {
+      const int rs = kc % kRawStages;
+      ok = mbar_wait(&raw_full[rs], (kc / kRawStages) & 1, P.err, 16);
+      if (!ok) break;
+      const uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
+      LaneWords L[2];
+      lds_lane_words<R>(raw, 2 * wq, lane, L[0]);
+      lds_lane_words<R>(raw, 2 * wq + 1, lane, L[1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&raw_empty[rs]);
+#define MATQ_SUBSTAGE(Q)                                                                       \
+      if (ok) {                                                                                \
+        const int i = kc * 4 + (Q), as = i % kAStages;                                         \
+        ok = mbar_wait(&a_empty[as], ((i / kAStages) & 1) ^ 1, P.err, 32);                     \
+        if (ok) {                                                                              \
+          const uint32_t a_slot = smem_u32(smem + S::kA + as * kATileBytes);                   \
+          dequant_substage<R, BN, GROUP, Q>(L, P, kc, rt0, wq, lane, a_slot);                  \
+          fence_proxy_async();                                                                 \
+          mbar_arrive(&a_full[as]);                                                            \
+        }                                                                                      \
+      }
+      MATQ_SUBSTAGE(0) MATQ_SUBSTAGE(1) MATQ_SUBSTAGE(2) MATQ_SUBSTAGE(3)
+#undef MATQ_SUBSTAGE
+    }
+    // epilogue: TMEM lanes 32*wq .. 32*wq+31 hold weight rows n0 + 32*wq + lane
+    if (ok) ok = mbar_wait(acc_full, 0, P.err, 64);
+    if (ok) {
+      tc_fence_after();
+      const int n = n0 + 32 * wq + lane;
+      const uint32_t taddr = tmem_d + ((uint32_t)(32 * wq) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (n < P.N) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int tok = m0 + c * 32 + i;
+            if (tok < P.M) {
+              const size_t o = (size_t)tok * P.N + n;
+              if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v[i]);
+              else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v[i];
+              else reinterpret_cast<float*>(P.y)[o] += v[i];
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"((uint32_t)BN) : "memory");
+  }
+}
+
+// ---- host side -----------------------------------------------------------------------------
+size_t prefill_workspace_bytes(int M, int K, int group) {
+  (void)group;
+  return ((((size_t)M * K * 2) + 255) & ~size_t(255)) + 256;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R, int BN, int GROUP>
+static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
+  using S = PrefillSmem<R, BN>;
+  auto kern = prefill_kernel<R, BN, GROUP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  if (e != cudaSuccess) return e;
+  dim3 grid((P.N + kBM - 1) / kBM, (P.M + BN - 1) / BN);
+  kern<<<grid, kThreads, S::kTotal, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], P);
+  return cudaGetLastError();
+}
+
+template <int BN, int GROUP>
+static cudaError_t launch_bn(int r, const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
+  switch (r) {
+    case 2: return launch_t<2, BN, GROUP>(maps, P, s);
+    case 3: return launch_t<3, BN, GROUP>(maps, P, s);
+    case 4: return launch_t<4, BN, GROUP>(maps, P, s);
+    case 6: return launch_t<6, BN, GROUP>(maps, P, s);
+    default: return launch_t<8, BN, GROUP>(maps, P, s);
+  }
+}
+
+cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g, const uint16_t* scales,
+                           const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
+                           cudaStream_t s) {
+  uint8_t* ws = (uint8_t*)workspace;
+  const size_t x16_bytes = (((size_t)M * K * 2) + 255) & ~size_t(255);
+  __half* x16 = (__half*)ws;
+  int* err = (int*)(ws + x16_bytes);
+  {
+    const size_t n = (size_t)M * K;
+    int blocks = (int)((n / 8 + 255) / 256);
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    xprep_prefill_kernel<<<blocks, 256, 0, s>>>((const uint16_t*)x, n, x16, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap maps[6];
+  const uint8_t* base = (const uint8_t*)planes;
+  for (int p = 0; p < kPlanes; ++p) {
+    const int b = plane_bits(p);
+    if (p < planes_for_width(r)) {
+      if (!make_map_2d(&maps[p], CU_TENSOR_MAP_DATA_TYPE_UINT64, base + g.off[p], (uint64_t)g.KC * b * 64,
+                       (uint64_t)g.RT, (uint64_t)g.KC * b * 512, (uint32_t)(b * 64), 8,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    } else {
+      maps[p] = maps[0];  // unused by this width
+    }
+  }
+  const int BN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  if (!make_map_2d(&maps[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
+                   (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  PrefillParams P;
+  P.M = M;
+  P.N = g.N;
+  P.K = K;
+  P.G = K / group;
+  P.RT = g.RT;
+  P.scales = scales;
+  P.zeros = zeros;
+  P.y = y;
+  P.y_mode = y_mode;
+  P.err = err;
+  if (group == 64) {
+    if (BN == 64) return launch_bn<64, 64>(r, maps, P, s);
+    if (BN == 128) return launch_bn<128, 64>(r, maps, P, s);
+    return launch_bn<256, 64>(r, maps, P, s);
+  }
+  if (BN == 64) return launch_bn<64, 128>(r, maps, P, s);
+  if (BN == 128) return launch_bn<128, 128>(r, maps, P, s);
+  return launch_bn<256, 128>(r, maps, P, s);
 }
 
 }  // namespace matq

@@ -141,3 +141,84 @@ def test_decode_full_size_sampled(M, shape, group):
             y = M.linear(dx, planes, 8, ds, dz, N, r, group).float().cpu().numpy()
             ref = O.linear(xv, q[rows], s[rows], z[rows], r, group)
             check_close(y[:, rows], ref, what=f"{shape} M={Mt} r={r}")
+
+
+# ---- prefill path ------------------------------------------------------------------------
+
+def _device_status(M, ws, Mt, K, N, group):
+    """The prefill path records a device-side status word (0 = ok) in the last 256 bytes
+    of the workspace."""
+    off = M.workspace_bytes(Mt, K, N, group) - 256
+    return int(ws[off:off + 4].cpu().numpy().view(np.int32)[0])
+
+
+@pytest.mark.parametrize("Mt,N,K,group", [(17, 128, 256, 128), (64, 200, 512, 64), (100, 384, 768, 128),
+                                          (129, 130, 512, 64), (300, 256, 1024, 128)])
+def test_prefill_small(M, Mt, N, K, group):
+    """Tiles of every token-tile size (64, 128, 256), ragged tokens and rows, both groups."""
+    import torch
+    q, s, z, xb, xv = problem(Mt, N, K, group, seed=Mt * 7 + N)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    ws = torch.empty(M.workspace_bytes(Mt, K, N, group), dtype=torch.uint8, device="cuda")
+    for r in O.WIDTHS:
+        ref = O.linear(xv, q, s, z, r, group)
+        for mode in (M.MATQ_OUT_BF16, M.MATQ_OUT_F32):
+            y = M.linear(dx, planes, 8, ds, dz, N, r, group, y_mode=mode, workspace=ws).float().cpu().numpy()
+            assert _device_status(M, ws, Mt, K, N, group) == 0
+            check_close(y, ref, what=f"M={Mt} N={N} K={K} g={group} r={r} mode={mode}")
+
+
+def test_prefill_accumulate_and_mode_a(M):
+    import torch
+    Mt, N, K = 40, 256, 512
+    q, s, z, xb, xv = problem(Mt, N, K, 128, seed=21)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    full = M.pack(dq, r_keep=8)
+    base = np.random.default_rng(2).standard_normal((Mt, N)).astype(np.float32)
+    y = torch.from_numpy(base.copy()).cuda()
+    M.linear(dx, full, 8, ds, dz, N, 4, 128, y=y, y_mode=M.MATQ_OUT_F32_ACCUM)
+    check_close(y.cpu().numpy(), base + O.linear(xv, q, s, z, 4, 128), what="accumulate")
+    for r in O.WIDTHS:
+        trunc = M.slice_copy(full, N, K, 8, r)
+        a = M.linear(dx, full, 8, ds, dz, N, r, 128, y_mode=M.MATQ_OUT_F32)
+        b = M.linear(dx, trunc, r, ds, dz, N, r, 128, y_mode=M.MATQ_OUT_F32)
+        assert torch.equal(a, b)
+
+
+def test_prefill_closed_forms(M):
+    N, K, Mt = 128, 512, 32
+    rng = np.random.default_rng(4)
+    z = rng.integers(0, 256, (N, K // 128), dtype=np.uint8)
+    q = np.repeat(z, 128, axis=1)
+    s = rng.uniform(1e-3, 1e-2, (N, K // 128)).astype(np.float16)
+    xb, xv = synth.bf16_round(rng.standard_normal((Mt, K)).astype(np.float32))
+    y = run(M, q, s, z, xb, 8, 128, y_mode=M.MATQ_OUT_F32)
+    assert np.all(y == 0.0)          # every weight dequantises to exactly 0 at r = 8
+
+
+@pytest.mark.parametrize("shape,group,Ms,widths", [
+    ((14336, 4096), 128, (2048,), (3, 4, 8)),
+    ((4096, 14336), 128, (2048,), (3, 4, 8)),
+    ((14336, 3584), 64, (32, 128, 512, 2048), (2, 3, 4, 6, 8)),
+    ((3584, 14336), 64, (32, 2048), (2, 8)),
+])
+def test_prefill_full_size_sampled(M, shape, group, Ms, widths):
+    """Benchmark shapes at the prefill batch sizes (8B FFN at M = 2048 with 1% outlier
+    channels x20; 9B FFN batch sweep), in the bench's launch configuration; 48 sampled output
+    rows against the oracle."""
+    import torch
+    N, K = shape
+    q, s, z = synth.parent_weights(N, K, group, seed=0, proj="gate" if N > K else "down")
+    dq = torch.from_numpy(q).cuda()
+    ds = torch.from_numpy(s.view(np.int16)).cuda()
+    dz = torch.from_numpy(z).cuda()
+    planes = M.pack(dq, r_keep=8)
+    rows = np.sort(np.random.default_rng(N + 1).choice(N, 48, replace=False))
+    for Mt in Ms:
+        xb, xv = synth.activations(Mt, K, seed=0, outlier_frac=0.01 if K == 4096 else 0.0)
+        dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        for r in widths:
+            y = M.linear(dx, planes, 8, ds, dz, N, r, group).float()[:, torch.from_numpy(rows).cuda()].cpu().numpy()
+            ref = O.linear(xv, q[rows], s[rows], z[rows], r, group)
+            check_close(y, ref, what=f"{shape} M={Mt} r={r}")
