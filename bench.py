@@ -276,7 +276,7 @@ def run_ours(args):
         xb, _ = synth.activations(M, D_MODEL, seed=rank, outlier_frac=spec["outlier"])
         xs[M] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
     Mmax = max(batches)
-    ws = torch.empty(max(matq.workspace_bytes(Mmax, D_FF, D_FF, GROUP), matq.workspace_bytes(Mmax, D_MODEL, D_FF, GROUP)),
+    ws = torch.zeros(max(matq.workspace_bytes(Mmax, D_FF, D_FF, GROUP), matq.workspace_bytes(Mmax, D_MODEL, D_FF, GROUP)),
                      dtype=torch.uint8, device=dev)
     gate_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
     up_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}

@@ -131,8 +131,22 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r,
 
 /* ---- the sliced linear layer ----------------------------------------------------------- */
 
-/* Workspace bytes matq_linear needs for these sizes (a multiple of 256). */
+/* Workspace bytes matq_linear needs for these sizes (a multiple of 256).
+ * A workspace starts with a fixed header (device status words and the counters that combine
+ * row groups split between CTAs).  The header must be zero-filled once before the first call
+ * (matq_workspace_init, or any zero fill); every successful call leaves it zero again, so a
+ * workspace is reused without re-initialisation.  Calls that share a workspace must be
+ * ordered on the device (one stream, or synchronised streams).  A workspace sized for
+ * (M_max, K_max, N) serves every call with M <= M_max and K <= K_max on either path. */
 size_t matq_linear_workspace(int M, int K, int N, int group);
+
+/* Zero the workspace header (asynchronous on `stream`).  ws_bytes: capacity of workspace. */
+int matq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronously read the device status left in the workspace header: 0 if every earlier call
+ * completed normally; otherwise the OR of internal wait-timeout codes (the outputs of the
+ * failing call are undefined; re-initialise the workspace before reusing it). */
+int matq_workspace_status(const void* workspace, int* status_out);
 
 /* y = x . W_hat_r^T for a width-r slice of a pack.
  *   x        [M, K] bf16, row-major, device.  Read only.
@@ -141,12 +155,14 @@ size_t matq_linear_workspace(int M, int K, int N, int group);
  *   y        [M, N] row-major, dtype by y_mode (MATQ_OUT_*).  MATQ_OUT_F32_ACCUM adds the
  *            product to the fp32 values already in y.
  *   workspace device scratch of >= matq_linear_workspace(M, K, N, group) bytes, owned by
- *            the caller; its contents need no initialisation and are clobbered.  Calls that
- *            share a workspace must be ordered (same stream, or synchronised).
- * Kernel choice is internal: M <= 16 takes the decode path (warp-level streaming GEMV /
- * skinny GEMM, fp32 accumulation); larger M the prefill path (TMA-staged planes,
- * dequantised to fp16 tiles in shared memory, tcgen05 MMA with TMEM accumulators).
- * The prefill path rounds x and W_hat to fp16; it needs |x| and |W_hat| below 65504. */
+ *            the caller, header zero-filled once (see matq_workspace_init).
+ * Kernel choice is internal: M <= 16 takes the decode path (persistent TMA-fed streaming
+ * kernel, weights unpacked in registers into exact fp16 MMA operands, fp32 accumulation;
+ * N <= 2^21); larger M the prefill path (TMA-staged planes dequantised to fp16 tiles in
+ * shared memory, tcgen05 MMA with TMEM accumulators).  The prefill path rounds x and W_hat
+ * to fp16; it needs |x| and |W_hat| below 65504.  Kernels are launched with programmatic
+ * dependent launch, so a call may start streaming weights while the previous kernel in the
+ * stream finishes; it reads x and writes y only after that kernel completes. */
 int matq_linear(const void* x, int M, int K,
                 const void* planes, int r_keep,
                 const uint16_t* scales, const uint8_t* zeros, int N,

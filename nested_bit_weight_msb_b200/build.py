@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmatq.so")
 SOURCES = ["api.cu", "pack.cu", "decode.cu", "prefill.cu", "glue.cu"]
-HEADERS = ["common.cuh", "internal.h", "operands.cuh"]
+HEADERS = ["common.cuh", "internal.h", "operands.cuh", "sync.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -116,9 +116,29 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r, void* p
 }
 
 size_t matq_linear_workspace(int M, int K, int N, int group) {
-  (void)N;
-  if (M < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
-  return M <= kDecodeMaxM ? decode_workspace_bytes(M, K, group) : prefill_workspace_bytes(M, K, group);
+  if (M < 1 || N < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
+  return M <= kDecodeMaxM ? decode_workspace_bytes(M) : workspace_header_bytes() + prefill_scratch_bytes(M, K);
+}
+
+int matq_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace) return MATQ_ENULL;
+  if (!aligned16(workspace)) return MATQ_EALIGN;
+  if (ws_bytes < workspace_header_bytes()) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(cudaMemsetAsync(workspace, 0, workspace_header_bytes(), (cudaStream_t)stream));
+}
+
+int matq_workspace_status(const void* workspace, int* status_out) {
+  if (!workspace || !status_out) return MATQ_ENULL;
+  if (!aligned16(workspace)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  int words[2] = {0, 0};
+  cudaError_t e = cudaMemcpy(words, workspace, sizeof(words), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e);
+  *status_out = words[0] | words[1];
+  return MATQ_OK;
 }
 
 int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
@@ -128,6 +148,7 @@ int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, con
   if (r > r_keep) return MATQ_ETRUNC;
   if (!valid_nk(N, K) || M < 1 || (long long)M * K > (1LL << 40) || (long long)M * N > (1LL << 40))
     return MATQ_EINVAL_SHAPE;
+  if (M <= kDecodeMaxM && (long long)N > max_decode_rows()) return MATQ_EINVAL_SHAPE;
   if (group != 64 && group != 128) return MATQ_EINVAL_GROUP;
   if (y_mode < MATQ_OUT_BF16 || y_mode > MATQ_OUT_F32_ACCUM) return MATQ_EDTYPE;
   if (!x || !planes || !scales || !zeros || !y || !workspace) return MATQ_ENULL;

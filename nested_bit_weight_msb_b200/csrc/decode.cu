@@ -1,236 +1,596 @@
-// Decode path (M <= 16): warp-level streaming skinny GEMM over the packed r-bit planes.
+// Decode path (M <= 16): one persistent, TMA-fed streaming kernel over the packed planes.
 //
-// Math (MatGPTQ App. A.1, delta folded into the zero point; MatGPTQ §4, Y = X W_D computed
-// as (W_D^T X^T)^T so that weights fill the 16-row MMA operand and tokens the 8-column one):
+// Math ("MatGPTQ: Efficient and Accurate Inference over Nested Quantized Models", App. A.1:
+// delta folded into the zero point; §4: Y = X W_D computed as (W_D^T X^T)^T so that the
+// weights fill the 16-row MMA operand and the tokens the 8-column one):
 //
 //   y[m, n] = sum_g s[n,g] * ( 2^(8-r) * sum_{k in g} x[m,k] * p[n,k]
 //                              + (delta_r - z[n,g]) * sum_{k in g} x[m,k] )
 //
-// Each warp owns a 16-row tile and a range of 256-input chunks.  It streams the planes of
-// width r with 16-byte-per-lane coalesced loads, turns the bits into fp16 MMA operand
-// registers in place (a mask-and-or against the fp16 bit pattern of 1024 gives 1024 + p*sigma
-// exactly, sigma a power of two fixed by the bit position), and feeds mma.sync m16n8k16 with
-// fp32 accumulation.  The per-position factors sigma are split into a per-row factor alpha
-// (folded into the group scale) and a per-input factor beta (folded into the activations:
-// inputs 8..15 of every 16-input MMA slice are pre-divided by 16 for r <= 4).  The 1024 bias
-// is removed per group with the exact sum Bs of the fp16 activation operands, and the zero
-// point term uses Sx, the plain per-group sum of x.  Per group, in fp32:
+// Operands.  A lane's plane words become fp16 A-operand registers in place: a mask-and-or
+// against the fp16 bit pattern of 1024 gives 1024 + sigma * v exactly (operands.cuh).  The
+// per-register powers of two sigma split into a per-row factor alpha (folded into the group
+// scale) and a per-input factor beta (inputs 8..15 of every 16-input MMA slice enter the B
+// operand divided by 16 for r <= 4, exact in fp16).  Two more MMAs per 16-input slice, with
+// constant A operands, accumulate the per-token sums the algebra needs in registers:
+// Dc = sum_k (-1024) * B_k (removes the 1024 bias) and Ds = sum_k beta_k * B_k = sum_k x_k
+// (the zero-point term).  Per 64-input slice of a group, in fp32:
 //
-//   y += a_row * (D - 1024 * Bs) + s * (delta_r - z) * Sx,   a_row = s * 2^(8-r) / alpha_row
+//   y += a_row * (D + Dc) + s * (delta_r - z) * Ds,   a_row = s * 2^(8-r) / alpha_row
 //
-// D is the fp32 MMA accumulator of that group.  No weight is ever rounded: the operands are
-// exact integers and x's fp16 operand equals x except below 2^-14 (fp16 subnormals).
+// Everything is linear in the inputs, so a group may be split between warps.  No weight is
+// ever rounded; x's fp16 operand equals x except below 2^-14 (fp16 subnormals).
+//
+// Schedule.  Work items are (row group of RG = 4 * RPW row tiles, 256-input chunk), ordered
+// row-group-major.  One persistent CTA per SM takes a balanced contiguous range of items
+// (stream-K style) and streams each into a shared-memory ring: the planes of width r (one
+// 2-D TMA per plane: exactly r bits per weight leave HBM), the chunk's bf16 activation rows
+// (one bulk copy per token into padded rows, so fragment loads are conflict-free) and the
+// rows' scales and zero points (cp.async).  Sixteen warps split each item 4 x 4: four row
+// slices of RPW row tiles times four 64-input slices; each warp reuses every activation
+// fragment across its row tiles.  Row groups inside a CTA's range are written directly.  A
+// row group split between CTAs is combined deterministically by its first contributor,
+// which works on it last: the others store their partial sums in their workspace slots and
+// count in; the first contributor waits (bounded) for the count and adds the slots in CTA
+// order.  The counters live in the workspace header; every call leaves them at zero.
+//
+// Launch.  Programmatic dependent launch: the kernel streams planes (which depend on no
+// earlier kernel) as soon as it is resident, and waits for the preceding kernel only before
+// reading activations or touching counters and y.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "operands.cuh"
+#include "sync.cuh"
 
 namespace matq {
 
-// ---- activation preparation ----------------------------------------------------------------
-// xfrag[(kt * NT + nt) * 32 + lane] = the m16n8k16 B-operand registers of lane `lane` for
-// input tile kt (16 inputs) and token tile nt (8 tokens): {x[t][k0], x[t][k0+1]} and
-// {x[t][k0+8], x[t][k0+9]} / beta_hi as fp16 pairs, t = 8*nt + lane/4, k0 = 16*kt + 2*(lane%4).
-// xsum[(g * NT*8 + t) * 2 + {0,1}] = {Bs, Sx}: sum over group g of the fp16 operands as used,
-// and sum of x.
-__device__ __forceinline__ float operand_value(const uint16_t* __restrict__ xrow, int k, float hi_scale) {
-  const float v = bf16_bits_to_float(xrow[k]);
-  const float sc = ((k & 15) >= 8) ? hi_scale : 1.0f;
-  return __half2float(__float2half_rn(v * sc));
-}
+constexpr int kRowSlices = 4;        // warps split an item's row tiles four ways ...
+// ... and its 256-input chunk into KSL = 2 slices of 128 inputs (8 warps, 256 threads: the
+// register budget of a thread stays at 255, and only two code variants share the I-cache)
+__host__ __device__ constexpr int k_slices(int NT) { return NT > 0 ? 2 : 2; }
+__host__ __device__ constexpr int dec_threads(int NT) { return 32 * kRowSlices * k_slices(NT); }
+constexpr int kDecStages = 4;        // ring depth
+constexpr int kMaxDecodeCTAs = 160;  // bound used to size the partial-sum workspace
+constexpr int kXPitch = kChunk * 2 + 16;  // bytes per activation row in a stage (padded)
 
-__global__ void xprep_decode_kernel(const uint16_t* __restrict__ x, int M, int K, int NT, int G, int group,
-                                    float hi_scale, uint2* __restrict__ xfrag, float* __restrict__ xsum,
-                                    int frag_blocks) {
-  if ((int)blockIdx.x < frag_blocks) {
-    const int KT = K / 16;
-    const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= (long long)KT * NT * 32) return;
-    const int lane = (int)(e & 31);
-    const int nt = (int)((e >> 5) % NT);
-    const int kt = (int)((e >> 5) / NT);
-    const int t = nt * 8 + (lane >> 2);
-    const int k0 = kt * 16 + 2 * (lane & 3);
-    uint2 out = make_uint2(0u, 0u);
-    if (t < M) {
-      const uint16_t* xr = x + (size_t)t * K;
-      __half2 lo = __floats2half2_rn(bf16_bits_to_float(xr[k0]), bf16_bits_to_float(xr[k0 + 1]));
-      __half2 hi = __floats2half2_rn(bf16_bits_to_float(xr[k0 + 8]) * hi_scale,
-                                     bf16_bits_to_float(xr[k0 + 9]) * hi_scale);
-      out.x = *reinterpret_cast<uint32_t*>(&lo);
-      out.y = *reinterpret_cast<uint32_t*>(&hi);
-    }
-    xfrag[e] = out;
-  } else {
-    const int NTOK = NT * 8;
-    const int e = (blockIdx.x - frag_blocks) * blockDim.x + threadIdx.x;
-    if (e >= G * NTOK) return;
-    const int g = e / NTOK, t = e % NTOK;
-    float bs = 0.f, sx = 0.f;
-    if (t < M) {
-      const uint16_t* xr = x + (size_t)t * K;
-      for (int k = g * group; k < (g + 1) * group; ++k) {
-        bs += operand_value(xr, k, hi_scale);
-        sx += bf16_bits_to_float(xr[k]);
-      }
-    }
-    xsum[2 * e] = bs;
-    xsum[2 * e + 1] = sx;
-  }
-}
+__host__ __device__ constexpr int rows_per_warp_tiles(int r) { return r <= 4 ? 4 : 2; }
 
-// ---- the kernel ------------------------------------------------------------------------------
 struct DecodeParams {
-  const uint8_t* planes;
-  PlaneGeom g;
+  int N, K, KC, RT, G, M, y_mode, C, NRG;
+  long long I;  // items
+  const uint16_t* x;
   const uint16_t* scales;
   const uint8_t* zeros;
-  int G;
-  const uint2* xfrag;
-  const float* xsum;
-  int M;
+  float* partial;
+  int* counters;
   void* y;
-  int y_mode;
-  int cpw;  // chunks per warp
+  int* err;
 };
 
 template <int R, int NT, int GROUP>
-__global__ void __launch_bounds__(256)
-decode_kernel(const DecodeParams P) {
-  constexpr int kBlocksPerGroup = GROUP / 32;
-  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
-  extern __shared__ float red[];  // [warps][NT*4][32]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  const int gid = lane >> 2, tg = lane & 3;
-  const int rt = blockIdx.x;
-  const PlaneGeom& g = P.g;
-  const int kc0 = warp * P.cpw;
-  const int kc1 = min(g.KC, kc0 + P.cpw);
+struct DecodeLayout {
+  static constexpr int RPW = rows_per_warp_tiles(R);
+  static constexpr int RG = kRowSlices * RPW;           // row tiles per item
+  static constexpr int NG = kChunk / GROUP;             // groups per chunk
+  static constexpr int NTOK = NT * 8;
+  static constexpr int kPlanes = RG * R * 512;          // all planes of width r for the item
+  static constexpr int kX = NTOK * kXPitch;             // activation rows of the chunk
+  static constexpr int kMetaS = RG * 16 * 8;            // per row: up to 4 fp16 scales (8 B)
+  static constexpr int kMetaZ = RG * 16 * 4;            // per row: one aligned 4-byte word of zeros
+  static constexpr int oX = kPlanes;
+  static constexpr int oS = oX + kX;
+  static constexpr int oZ = oS + kMetaS;
+  static constexpr int kStage = ((oZ + kMetaZ) + 127) & ~127;
+  static constexpr int KSL = k_slices(NT);
+  static constexpr int kThreads = dec_threads(NT);
+  static constexpr int oRed = kDecStages * kStage;     // k-slice reduction buffer
+  static constexpr int kRed = (KSL - 1) * kRowSlices * RPW * NT * 4 * 32 * 4;
+  static constexpr int oBar = oRed + kRed;
+  static constexpr int kSmem = oBar + 2 * kDecStages * 8 + 128;
+};
 
-  // per-row promotion factors: a = s * 2^(8-r) / alpha_row
+// plane p's offset inside an item's plane region (RG row tiles each)
+template <int RG>
+__device__ __forceinline__ int item_plane_off(int p) {
+  return RG * 512 * (p == 0 ? 0 : p == 1 ? 2 : p == 2 ? 3 : p == 3 ? 4 : 6);
+}
+
+// Lane words of the NB blocks NB*KS .. NB*KS+NB-1 of row tile t (at their natural indices).
+template <int R, int RG, int NB, int KS>
+__device__ __forceinline__ void lds_slice_words(const uint8_t* planes, int t, int lane, LaneWords& L) {
+  constexpr int w0 = NB * KS;                             // first block of the slice
+  constexpr int half = w0 / 4, wo = (w0 % 4) * 4;         // 2-bit planes: 512-byte half, byte offset
+  auto two_bit = [&](int p, uint32_t* dst) {
+    const uint8_t* src = planes + item_plane_off<RG>(p) + t * 1024 + half * 512 + lane * 16 + wo;
+    if constexpr (NB == 4) {
+      const uint4 a = *reinterpret_cast<const uint4*>(src);
+      dst[w0] = a.x; dst[w0 + 1] = a.y; dst[w0 + 2] = a.z; dst[w0 + 3] = a.w;
+    } else {
+      const uint2 a = *reinterpret_cast<const uint2*>(src);
+      dst[w0] = a.x; dst[w0 + 1] = a.y;
+    }
+  };
+  auto one_bit = [&](int p, uint32_t* dst) {
+    const uint8_t* src = planes + item_plane_off<RG>(p) + t * 512 + lane * 16 + (w0 / 2) * 4;
+    if constexpr (NB == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(src);
+      dst[w0 / 2] = a.x; dst[w0 / 2 + 1] = a.y;
+    } else {
+      dst[w0 / 2] = *reinterpret_cast<const uint32_t*>(src);
+    }
+  };
+  two_bit(0, L.p0);
+  if constexpr (R >= 3) one_bit(1, L.p1);
+  if constexpr (R >= 4) one_bit(2, L.p2);
+  if constexpr (R >= 6) two_bit(3, L.p3);
+  if constexpr (R >= 8) two_bit(4, L.p4);
+}
+
+// B-operand registers of one 16-input MMA slice (inputs k0..k0+15 of the chunk) for token
+// tile nt, built from the bf16 activation rows in the stage: {x[k], x[k+1]} and
+// {x[k+8], x[k+9]} * hi_scale as fp16 pairs, k = k0 + 2*(lane%4), token 8*nt + lane/4.
+__device__ __forceinline__ void b_frag(const uint8_t* xs, int nt, int k0, int lane, float hi_scale, uint32_t& b0,
+                                       uint32_t& b1) {
+  const uint8_t* row = xs + (nt * 8 + (lane >> 2)) * kXPitch + (k0 + 2 * (lane & 3)) * 2;
+  const uint32_t lo = *reinterpret_cast<const uint32_t*>(row);
+  const uint32_t hi = *reinterpret_cast<const uint32_t*>(row + 16);
+  __half2 l = __floats2half2_rn(__uint_as_float(lo << 16), __uint_as_float(lo & 0xFFFF0000u));
+  __half2 h = __floats2half2_rn(__uint_as_float(hi << 16) * hi_scale, __uint_as_float(hi & 0xFFFF0000u) * hi_scale);
+  b0 = *reinterpret_cast<uint32_t*>(&l);
+  b1 = *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ long long item_begin(long long c, long long I, long long C) { return c * I / C; }
+// CTA whose range holds item u (every CTA has at least one item: C <= I)
+__device__ __forceinline__ long long item_owner(long long u, long long I, long long C) {
+  return ((u + 1) * C - 1) / I;
+}
+
+// Work of one warp: RPW row tiles (row slice rs) x input slice KS of every item.
+template <int R, int NT, int GROUP, int KS, typename Refill>
+__device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                                            float* red, long long c, long long ib, long long ie, int rs, int lane,
+                                            Refill&& refill) {
+  using Lt = DecodeLayout<R, NT, GROUP>;
+  constexpr int RPW = Lt::RPW, RG = Lt::RG, NG = Lt::NG, KSL = Lt::KSL;
+  constexpr int NB = 8 / KSL;                                    // 32-input blocks per slice
+  constexpr int kPromoteEvery = (GROUP / 32 < NB) ? GROUP / 32 : NB;  // blocks per scale group part
+  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
+  constexpr float kHiScale = (R <= 4) ? 0.0625f : 1.0f;
+  // constant A operands: -1024 everywhere (bias removal) and beta per input (token sums)
+  constexpr uint32_t kNeg1024 = 0xE400E400u;
+  constexpr uint32_t kOne = 0x3C003C00u, kBetaHi = (R <= 4) ? 0x4C004C00u : 0x3C003C00u;  // 1.0, 16.0
+  constexpr int kLaneFloats = RPW * NT * 4;
+  constexpr int kSlotFloats = kLaneFloats * 32;
+  const int gid = lane >> 2, tg = lane & 3;
+  const int nitems = (int)(ie - ib);
   float amul[2];
   if constexpr (R == 2) { amul[0] = 64.f; amul[1] = 16.f; }
   else if constexpr (R == 3) { amul[0] = amul[1] = 32.f; }
   else if constexpr (R == 4) { amul[0] = amul[1] = 16.f; }
   else { amul[0] = amul[1] = 1.f; }
-  const int row0 = rt * kTileRows + gid, row1 = row0 + 8;
-  const bool v0 = row0 < g.N, v1 = row1 < g.N;
+  const uint32_t Ac[4] = {kNeg1024, kNeg1024, kNeg1024, kNeg1024};
+  const uint32_t As[4] = {kOne, kOne, kBetaHi, kBetaHi};
 
-  float yacc[NT][4];
+  float yacc[RPW][NT][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) yacc[nt][i] = 0.f;
-
-  bool bvalid[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) bvalid[nt] = (nt * 8 + gid) < P.M;
-
-  for (int kc = kc0; kc < kc1; ++kc) {
-    LaneWords L;
-    load_lane_words<R>(P.planes, g, (size_t)rt * g.KC + kc, lane, L);
-    uint2 bfr[16][NT];
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        bfr[i][nt] = bvalid[nt] ? __ldg(&P.xfrag[((size_t)(kc * 16 + i) * NT + nt) * 32 + lane]) : make_uint2(0u, 0u);
-
-    float d[NT][4];
+  for (int j = 0; j < RPW; ++j)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) d[nt][i] = 0.f;
+      for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
 
-#define MATQ_BLOCK(W)                                                                  \
-    {                                                                                  \
-      uint32_t A[2][4];                                                                \
-      build_operands<R, W>(L, A);                                                      \
-      _Pragma("unroll") for (int j = 0; j < 2; ++j)                                    \
-      _Pragma("unroll") for (int nt = 0; nt < NT; ++nt)                                \
-        mma_f16(d[nt], A[j], bfr[2 * (W) + j][nt].x, bfr[2 * (W) + j][nt].y);          \
-      if (((W) + 1) % kBlocksPerGroup == 0) {                                          \
-        const int gi = (kc * kChunk + 32 * ((W) + 1)) / GROUP - 1;                     \
-        promote(gi, d);                                                                \
-      }                                                                                \
+  bool ok = true;
+  for (int n = 0; n < nitems; ++n) {
+    const int s = n % kDecStages;
+    const long long it = ib + n;
+    const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
+    if (ok) ok = mbar_wait(&full[s], (n / kDecStages) & 1, P.err, 2);
+    if (ok) {
+      const uint8_t* st = smem + s * Lt::kStage;
+      LaneWords L[RPW];
+#pragma unroll
+      for (int j = 0; j < RPW; ++j) lds_slice_words<R, RG, NB, KS>(st, rs * RPW + j, lane, L[j]);
+
+      float d[RPW][NT][4], dc[NT][4], ds[NT][4];
+      auto zero_acc = [&]() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            dc[nt][i] = 0.f;
+            ds[nt][i] = 0.f;
+#pragma unroll
+            for (int j = 0; j < RPW; ++j) d[j][nt][i] = 0.f;
+          }
+      };
+      // fold the inputs accumulated so far (all in scale group gl) into the running sums
+      auto promote = [&](int gl) {
+#pragma unroll
+        for (int j = 0; j < RPW; ++j) {
+          float a[2], cz[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int rr = (rs * RPW + j) * 16 + gid + 8 * h;  // row inside the item
+            const int row = rg * RG * 16 + rr;
+            float sv = 0.f, zv = 0.f;
+            if (row < P.N) {
+              sv = __half2float(*reinterpret_cast<const __half*>(st + Lt::oS + rr * 8 + gl * 2));
+              const int zoff = (int)(((size_t)row * P.G + (size_t)kc * NG) & 3);
+              zv = (float)st[Lt::oZ + rr * 4 + zoff + gl];
+            }
+            a[h] = sv * amul[h];
+            cz[h] = sv * (kDelta - zv);
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              yacc[j][nt][i] = fmaf(cz[i >> 1], ds[nt][i], fmaf(a[i >> 1], d[j][nt][i] + dc[nt][i], yacc[j][nt][i]));
+        }
+        zero_acc();
+      };
+      zero_acc();
+
+#pragma unroll
+      for (int wb = 0; wb < NB; ++wb) {
+        uint32_t b0[2][NT], b1[2][NT];
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            b_frag(st + Lt::oX, nt, (NB * KS + wb) * 32 + 16 * jj, lane, kHiScale, b0[jj][nt], b1[jj][nt]);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16(dc[nt], Ac, b0[jj][nt], b1[jj][nt]);
+            mma_f16(ds[nt], As, b0[jj][nt], b1[jj][nt]);
+          }
+#pragma unroll
+        for (int j = 0; j < RPW; ++j) {
+          uint32_t A[2][4];
+          build_slice_operands<R, NB * KS>(L[j], wb, A);
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_f16(d[j][nt], A[jj], b0[jj][nt], b1[jj][nt]);
+        }
+        if ((wb + 1) % kPromoteEvery == 0) promote(((NB * KS + wb) * 32) / GROUP);
+      }
     }
-    auto promote = [&](int gi, float (&dd)[NT][4]) {
-      float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
-      if (v0) {
-        const float s = __half2float(__ushort_as_half(P.scales[(size_t)row0 * P.G + gi]));
-        a0 = s * amul[0];
-        c0 = s * (kDelta - (float)P.zeros[(size_t)row0 * P.G + gi]);
-      }
-      if (v1) {
-        const float s = __half2float(__ushort_as_half(P.scales[(size_t)row1 * P.G + gi]));
-        a1 = s * amul[1];
-        c1 = s * (kDelta - (float)P.zeros[(size_t)row1 * P.G + gi]);
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float4 xs = *reinterpret_cast<const float4*>(P.xsum + ((size_t)gi * NT * 8 + nt * 8 + 2 * tg) * 2);
-        // xs = {Bs(t0), Sx(t0), Bs(t1), Sx(t1)}
-        yacc[nt][0] = fmaf(c0, xs.y, fmaf(a0, fmaf(-1024.f, xs.x, dd[nt][0]), yacc[nt][0]));
-        yacc[nt][1] = fmaf(c0, xs.w, fmaf(a0, fmaf(-1024.f, xs.z, dd[nt][1]), yacc[nt][1]));
-        yacc[nt][2] = fmaf(c1, xs.y, fmaf(a1, fmaf(-1024.f, xs.x, dd[nt][2]), yacc[nt][2]));
-        yacc[nt][3] = fmaf(c1, xs.w, fmaf(a1, fmaf(-1024.f, xs.z, dd[nt][3]), yacc[nt][3]));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dd[nt][i] = 0.f;
-      }
-    };
-    MATQ_BLOCK(0) MATQ_BLOCK(1) MATQ_BLOCK(2) MATQ_BLOCK(3)
-    MATQ_BLOCK(4) MATQ_BLOCK(5) MATQ_BLOCK(6) MATQ_BLOCK(7)
-#undef MATQ_BLOCK
-  }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    // the streaming warps (0..7) refill this slot with item n + S once every warp released it
+    if (rs + kRowSlices * KS < 8 && n + kDecStages < nitems && ok) {
+      ok = mbar_wait(&empty[s], (n / kDecStages) & 1, P.err, 1);
+      if (ok) refill(n + kDecStages);
+    }
 
-  // reduce the warps' partial sums (fixed order) and store
+    // flush at the end of a row group (or of this CTA's range); all warps get here for the
+    // same items, so the four k-slices of a row slice meet at a named barrier
+    if (n == nitems - 1 || (it + 1) / P.KC != rg) {
+      const long long g0 = (long long)rg * P.KC, g1 = g0 + P.KC;
+      const bool whole = g0 >= ib && g1 <= ie;
+      if (KS > 0) {
+        float4* mine =
+            reinterpret_cast<float4*>(red + ((KS - 1) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+        for (int j = 0; j < RPW; ++j)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) red[((warp * NT + nt) * 4 + i) * 32 + lane] = yacc[nt][i];
-  __syncthreads();
-  if (warp == 0) {
+          for (int nt = 0; nt < NT; ++nt)
+            mine[j * NT + nt] = make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
+      if (KS == 0) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+        for (int k2 = 0; k2 < KSL - 1; ++k2) {
+          const float4* o = reinterpret_cast<const float4*>(red + (k2 * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float v = 0.f;
-        for (int w = 0; w < nwarps; ++w) v += red[((w * NT + nt) * 4 + i) * 32 + lane];
-        const int row = (i < 2) ? row0 : row1;
-        const int tok = nt * 8 + 2 * tg + (i & 1);
-        if (row < g.N && tok < P.M) {
-          const size_t o = (size_t)tok * g.N + row;
-          if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
-          else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v;
-          else reinterpret_cast<float*>(P.y)[o] += v;
+          for (int j = 0; j < RPW; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float4 v = o[j * NT + nt];
+              yacc[j][nt][0] += v.x;
+              yacc[j][nt][1] += v.y;
+              yacc[j][nt][2] += v.z;
+              yacc[j][nt][3] += v.w;
+            }
+        }
+        auto store_y = [&](int j, int nt, int i, float v) {
+          const int row = (rg * RG + rs * RPW + j) * 16 + gid + 8 * (i >> 1);
+          const int tok = nt * 8 + 2 * tg + (i & 1);
+          if (row < P.N && tok < P.M) {
+            const size_t o = (size_t)tok * P.N + row;
+            if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
+            else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v;
+            else reinterpret_cast<float*>(P.y)[o] += v;
+          }
+        };
+        if (whole) {
+#pragma unroll
+          for (int j = 0; j < RPW; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) store_y(j, nt, i, yacc[j][nt][i]);
+        } else if (ok) {
+          // Split row group: its first contributor c_first works on it last (its items end
+          // c_first's range and start everybody else's), so c_first combines; the others
+          // store their partial sums and count in.
+          const long long cf = item_owner(g0, P.I, P.C), cl = item_owner(g1 - 1, P.I, P.C);
+          int* cnt = &P.counters[rg * kRowSlices + rs];
+          if (c != cf) {
+            const int side = (rg == (int)(ib / P.KC)) ? 0 : 1;
+            float4* mine = reinterpret_cast<float4*>(
+                P.partial + ((size_t)(c * 2 + side) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+#pragma unroll
+            for (int j = 0; j < RPW; ++j)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                __stcg(&mine[j * NT + nt], make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]));
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(cnt, 1);
+          } else {
+            bool arrived = true;
+            if (lane == 0) {
+              const int want = (int)(cl - cf);
+              const long long t0 = clock64();
+              while (atomicAdd(cnt, 0) < want) {
+                if (clock64() - t0 > kWaitCycles) {
+                  atomicOr(P.err, 128);
+                  arrived = false;
+                  break;
+                }
+                __nanosleep(64);
+              }
+              atomicExch(cnt, 0);  // leave the counter at zero for the next call
+            }
+            arrived = __shfl_sync(0xffffffffu, arrived ? 1 : 0, 0) != 0;
+            __threadfence();
+            float4 acc[RPW * NT];
+#pragma unroll
+            for (int j = 0; j < RPW; ++j)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                acc[j * NT + nt] = make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
+            // the other contributors in CTA order (deterministic); kU at a time so loads overlap
+            constexpr int kU = (RPW * NT >= 8) ? 2 : (16 / (RPW * NT));
+            for (long long c2 = cf + 1; arrived && c2 <= cl; c2 += kU) {
+              float4 v[kU][RPW * NT];
+#pragma unroll
+              for (int u = 0; u < kU; ++u) {
+                if (c2 + u <= cl) {
+                  const long long cc = c2 + u;
+                  const int side2 = (rg == (int)(item_begin(cc, P.I, P.C) / P.KC)) ? 0 : 1;
+                  const float4* src = reinterpret_cast<const float4*>(
+                      P.partial + ((size_t)(cc * 2 + side2) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+#pragma unroll
+                  for (int q = 0; q < RPW * NT; ++q) v[u][q] = __ldcg(&src[q]);
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < kU; ++u)
+                if (c2 + u <= cl)
+#pragma unroll
+                  for (int q = 0; q < RPW * NT; ++q) {
+                    acc[q].x += v[u][q].x;
+                    acc[q].y += v[u][q].y;
+                    acc[q].z += v[u][q].z;
+                    acc[q].w += v[u][q].w;
+                  }
+            }
+#pragma unroll
+            for (int j = 0; j < RPW; ++j)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                store_y(j, nt, 0, acc[j * NT + nt].x);
+                store_y(j, nt, 1, acc[j * NT + nt].y);
+                store_y(j, nt, 2, acc[j * NT + nt].z);
+                store_y(j, nt, 3, acc[j * NT + nt].w);
+              }
+          }
         }
       }
+      // the reduction buffer may be overwritten only after the k-slice-0 warps have read it
+      asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
+#pragma unroll
+      for (int j = 0; j < RPW; ++j)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
+    }
   }
-}
-
-// ---- host launch ---------------------------------------------------------------------------
-size_t decode_workspace_bytes(int M, int K, int group) {
-  const int NT = (M <= 8) ? 1 : 2;
-  const size_t frag = (size_t)(K / 16) * NT * 32 * sizeof(uint2);
-  const size_t sums = (size_t)(K / group) * NT * 8 * 2 * sizeof(float);
-  return ((frag + 255) & ~size_t(255)) + ((sums + 255) & ~size_t(255));
 }
 
 template <int R, int NT, int GROUP>
-static cudaError_t launch_decode_t(const DecodeParams& P, int warps, cudaStream_t s) {
-  const size_t smem = (size_t)warps * NT * 4 * 32 * sizeof(float);
-  decode_kernel<R, NT, GROUP><<<P.g.RT, warps * 32, smem, s>>>(P);
-  return cudaGetLastError();
+__global__ void __launch_bounds__(dec_threads(NT), 1)
+decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+              const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tm3,
+              const __grid_constant__ CUtensorMap tm4, const DecodeParams P) {
+  using Lt = DecodeLayout<R, NT, GROUP>;
+  constexpr int RG = Lt::RG, NG = Lt::NG, NTOK = Lt::NTOK;
+  constexpr int kNumPlanes = planes_for_width(R);
+  constexpr int kThreads = Lt::kThreads;
+  constexpr int kStreamers = 256;  // threads of warps 0..7, which refill the ring
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lt::oBar);
+  uint64_t* empty = full + kDecStages;
+  float* red = reinterpret_cast<float*>(smem + Lt::oRed);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long c = blockIdx.x;
+  const long long ib = item_begin(c, P.I, P.C), ie = item_begin(c + 1, P.I, P.C);
+  const int nitems = (int)(ie - ib);
+  const CUtensorMap* maps[5] = {&tm0, &tm1, &tm2, &tm3, &tm4};
+  const int mrows = P.M < NTOK ? P.M : NTOK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&full[s], 1 + kStreamers);  // thread 0's arrival + one arrival per streamer
+      mbar_init(&empty[s], kThreads / 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // activation rows >= M stay zero in every stage (nothing is ever copied there)
+  for (int s = 0; s < kDecStages; ++s)
+    for (int i = threadIdx.x; i < (NTOK - mrows) * kXPitch / 4; i += kThreads)
+      reinterpret_cast<uint32_t*>(smem + s * Lt::kStage + Lt::oX + mrows * kXPitch)[i] = 0u;
+  __syncthreads();
+  // the next kernel in the stream may launch its prologue now
+  pdl_launch_dependents();
+
+  // Planes of item n into slot n % S (2-D TMA by thread 0): they depend on no earlier kernel.
+  auto stream_planes = [&](int n) {
+    if (threadIdx.x == 0) {
+      const int s = n % kDecStages;
+      const long long it = ib + n;
+      const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
+      uint8_t* st = smem + s * Lt::kStage;
+      mbar_expect_tx_only(&full[s], Lt::kPlanes + mrows * kChunk * 2);
+#pragma unroll
+      for (int p = 0; p < kNumPlanes; ++p)
+        tma_load_2d(st + item_plane_off<RG>(p), maps[p], kc * plane_bits(p) * 64, rg * RG, &full[s]);
+    }
+  };
+  // Activation rows (a bulk copy per token), scales and zero points (cp.async, one row per
+  // streamer thread) of item n; called by the streamer threads (warps 0..7) only.
+  auto stream_rest = [&](int n) {
+    const int s = n % kDecStages;
+    const long long it = ib + n;
+    const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
+    uint8_t* st = smem + s * Lt::kStage;
+    const int t = threadIdx.x;
+    if (t < mrows) bulk_load(st + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk, kChunk * 2, &full[s]);
+    // scales (NG fp16) and the aligned 4-byte word of zeros holding this chunk's NG bytes.
+    // The word never crosses the end of the zeros array except when its NG = 2 bytes are the
+    // array's last two and start a word; that row is copied with a plain 2-byte load.
+    const int row = rg * RG * 16 + t;
+    bool plain = false;
+    if (t < RG * 16 && row < P.N) {
+      const uint16_t* sp = P.scales + (size_t)row * P.G + (size_t)kc * NG;
+      if constexpr (NG == 2) cp_async4(st + Lt::oS + t * 8, sp);
+      else cp_async8(st + Lt::oS + t * 8, sp);
+      const size_t zi = (size_t)row * P.G + (size_t)kc * NG;
+      if ((zi & 3) == 0 && zi + 4 > (size_t)P.N * P.G) {
+        plain = true;
+        *reinterpret_cast<uint16_t*>(st + Lt::oZ + t * 4) = *reinterpret_cast<const uint16_t*>(P.zeros + zi);
+      } else {
+        cp_async4(st + Lt::oZ + t * 4, P.zeros + (zi & ~(size_t)3));
+      }
+    }
+    if (plain) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      mbar_arrive(&full[s]);  // a plain arrive releases the plain store too
+    } else {
+      cp_async_arrive_noinc(&full[s]);
+    }
+    if (t == 0) mbar_arrive(&full[s]);
+  };
+  auto refill = [&](int n) {
+    stream_planes(n);
+    stream_rest(n);
+  };
+
+  const int pre = nitems < kDecStages ? nitems : kDecStages;
+  for (int n = 0; n < pre; ++n) stream_planes(n);
+  pdl_wait();  // activations, counters and y belong to earlier kernels in the stream
+  if (warp < 8)
+    for (int n = 0; n < pre; ++n) stream_rest(n);
+
+  const int rs = warp & 3, ks = warp >> 2;
+  if constexpr (Lt::KSL == 2) {
+    if (ks == 0) decode_warp<R, NT, GROUP, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+    else decode_warp<R, NT, GROUP, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+    return;
+  }
+  switch (ks) {
+    case 0: decode_warp<R, NT, GROUP, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
+    case 1: decode_warp<R, NT, GROUP, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
+    case 2: decode_warp<R, NT, GROUP, 2>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
+    default: decode_warp<R, NT, GROUP, 3>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
+  }
+}
+
+// ---- host side -----------------------------------------------------------------------------
+// Workspace: [header: error word + split-row-group counters, zero-filled once by the caller
+// and left zero by every call][decode partial-sum slots | prefill scratch].
+constexpr size_t kHeaderCounters = size_t(1) << 16;
+constexpr size_t kHeaderBytes = 256 + kHeaderCounters * sizeof(int);
+
+size_t workspace_header_bytes() { return kHeaderBytes; }
+long long max_decode_rows() { return (long long)(kHeaderCounters / kRowSlices) * 8 * kTileRows; }
+
+size_t decode_workspace_bytes(int M) {
+  const int NT = (M <= 8) ? 1 : 2;
+  const size_t partial = (size_t)2 * kMaxDecodeCTAs * kRowSlices * 4 * NT * 4 * 32 * sizeof(float);
+  return kHeaderBytes + ((partial + 255) & ~size_t(255));
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+static cudaError_t plane_map(CUtensorMap* m, const uint8_t* base, const PlaneGeom& g, int p, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const int b = plane_bits(p);
+  const cuuint64_t dims[2] = {(cuuint64_t)g.KC * b * 64, (cuuint64_t)g.RT};
+  const cuuint64_t strides[1] = {(cuuint64_t)g.KC * b * 512};
+  const cuuint32_t box[2] = {(cuuint32_t)(b * 64), (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base + g.off[p]), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int R, int NT, int GROUP>
+static cudaError_t launch_decode_t(const uint8_t* planes, const PlaneGeom& g, DecodeParams P, int sms,
+                                   cudaStream_t s) {
+  using Lt = DecodeLayout<R, NT, GROUP>;
+  CUtensorMap maps[5];
+  for (int p = 0; p < 5; ++p) {
+    if (p < planes_for_width(R)) {
+      cudaError_t e = plane_map(&maps[p], planes, g, p, Lt::RG);
+      if (e != cudaSuccess) return e;
+    } else {
+      maps[p] = maps[0];
+    }
+  }
+  P.NRG = (g.RT + Lt::RG - 1) / Lt::RG;
+  P.I = (long long)P.NRG * g.KC;
+  P.C = (int)(P.I < sms ? P.I : sms);
+  auto kern = decode_kernel<R, NT, GROUP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(P.C), dim3(Lt::kThreads), (size_t)Lt::kSmem, s, maps[0], maps[1], maps[2], maps[3],
+                    maps[4], P);
 }
 
 template <int NT, int GROUP>
-static cudaError_t launch_decode_r(int r, const DecodeParams& P, int warps, cudaStream_t s) {
+static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom& g, const DecodeParams& P, int sms,
+                                   cudaStream_t s) {
   switch (r) {
-    case 2: return launch_decode_t<2, NT, GROUP>(P, warps, s);
-    case 3: return launch_decode_t<3, NT, GROUP>(P, warps, s);
-    case 4: return launch_decode_t<4, NT, GROUP>(P, warps, s);
-    case 6: return launch_decode_t<6, NT, GROUP>(P, warps, s);
-    default: return launch_decode_t<8, NT, GROUP>(P, warps, s);
+    case 2: return launch_decode_t<2, NT, GROUP>(planes, g, P, sms, s);
+    case 3: return launch_decode_t<3, NT, GROUP>(planes, g, P, sms, s);
+    case 4: return launch_decode_t<4, NT, GROUP>(planes, g, P, sms, s);
+    case 6: return launch_decode_t<6, NT, GROUP>(planes, g, P, sms, s);
+    default: return launch_decode_t<8, NT, GROUP>(planes, g, P, sms, s);
   }
 }
 
@@ -238,41 +598,30 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
                           const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
                           cudaStream_t s) {
   const int NT = (M <= 8) ? 1 : 2;
-  const int G = K / group;
   uint8_t* ws = (uint8_t*)workspace;
-  const size_t frag = (size_t)(K / 16) * NT * 32 * sizeof(uint2);
-  uint2* xfrag = (uint2*)ws;
-  float* xsum = (float*)(ws + ((frag + 255) & ~size_t(255)));
-  const float hi_scale = (r <= 4) ? 0.0625f : 1.0f;
-  {
-    const int threads = 256;
-    const long long nfrag = (long long)(K / 16) * NT * 32;
-    const int fb = (int)((nfrag + threads - 1) / threads);
-    const int sb = (G * NT * 8 + threads - 1) / threads;
-    xprep_decode_kernel<<<fb + sb, threads, 0, s>>>((const uint16_t*)x, M, K, NT, G, group, hi_scale, xfrag, xsum,
-                                                    fb);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms > kMaxDecodeCTAs) sms = kMaxDecodeCTAs;
   DecodeParams P;
-  P.planes = (const uint8_t*)planes;
-  P.g = g;
+  P.N = g.N;
+  P.K = K;
+  P.KC = g.KC;
+  P.RT = g.RT;
+  P.G = K / group;
+  P.M = M;
+  P.y_mode = y_mode;
+  P.x = (const uint16_t*)x;
   P.scales = scales;
   P.zeros = zeros;
-  P.G = G;
-  P.xfrag = xfrag;
-  P.xsum = xsum;
-  P.M = M;
+  P.err = (int*)ws;
+  P.counters = (int*)(ws + 256);
+  P.partial = (float*)(ws + kHeaderBytes);
   P.y = y;
-  P.y_mode = y_mode;
-  int warps = g.KC >= 8 ? 8 : g.KC;
-  P.cpw = (g.KC + warps - 1) / warps;
-  warps = (g.KC + P.cpw - 1) / P.cpw;
-  if (NT == 1) {
-    return group == 64 ? launch_decode_r<1, 64>(r, P, warps, s) : launch_decode_r<1, 128>(r, P, warps, s);
-  } else {
-    return group == 64 ? launch_decode_r<2, 64>(r, P, warps, s) : launch_decode_r<2, 128>(r, P, warps, s);
-  }
+  const uint8_t* pl = (const uint8_t*)planes;
+  if (NT == 1)
+    return group == 64 ? launch_decode_r<1, 64>(r, pl, g, P, sms, s) : launch_decode_r<1, 128>(r, pl, g, P, sms, s);
+  return group == 64 ? launch_decode_r<2, 64>(r, pl, g, P, sms, s) : launch_decode_r<2, 128>(r, pl, g, P, sms, s);
 }
 
 }  // namespace matq

@@ -5,11 +5,14 @@
 // are HBM-bound elementwise passes with fp32 arithmetic and bf16 outputs.
 #include "common.cuh"
 #include "internal.h"
+#include "sync.cuh"
 
 namespace matq {
 
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ h, int D, float eps,
                                                       __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x;
   const float* hr = h + (size_t)row * D;
   float ss = 0.f;
@@ -31,6 +34,8 @@ __device__ __forceinline__ float silu_f(float t) { return t / (1.0f + expf(-t));
 __global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __restrict__ gate,
                                                        const __nv_bfloat16* __restrict__ up, size_t n,
                                                        __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t nvec = n / 8;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
@@ -52,8 +57,7 @@ __global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __re
 }
 
 cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s) {
-  rmsnorm_kernel<<<M, 256, 0, s>>>(h, D, eps, (__nv_bfloat16*)out);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_kernel, dim3(M), dim3(256), 0, s, h, D, eps, (__nv_bfloat16*)out);
 }
 
 cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s) {
@@ -62,9 +66,8 @@ cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void
   int blocks = (int)((nvec + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  silu_mul_kernel<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)gate, (const __nv_bfloat16*)up, n,
-                                         (__nv_bfloat16*)out);
-  return cudaGetLastError();
+  return launch_pdl(silu_mul_kernel, dim3(blocks), dim3(256), 0, s, (const __nv_bfloat16*)gate,
+                    (const __nv_bfloat16*)up, n, (__nv_bfloat16*)out);
 }
 
 }  // namespace matq

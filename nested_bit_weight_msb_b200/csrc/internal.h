@@ -9,12 +9,16 @@ namespace matq {
 cudaError_t launch_pack(const uint8_t* codes, const PlaneGeom& g, int r_keep, void* planes, cudaStream_t s);
 cudaError_t launch_slice(const void* planes, const PlaneGeom& g, int r, uint8_t* out, cudaStream_t s);
 
-size_t decode_workspace_bytes(int M, int K, int group);
+// Workspace = [header: device error words + split-row-group counters; zero-filled once by the
+// caller, left zero by every call][scratch of the path taken].
+size_t workspace_header_bytes();
+long long max_decode_rows();
+size_t decode_workspace_bytes(int M);  // header included
 cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
                           const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
                           int y_mode, void* workspace, cudaStream_t s);
 
-size_t prefill_workspace_bytes(int M, int K, int group);
+size_t prefill_scratch_bytes(int M, int K);  // after the header
 cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
                            const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
                            int y_mode, void* workspace, cudaStream_t s);

@@ -124,4 +124,15 @@ __device__ __forceinline__ void build_operands(const LaneWords& L, uint32_t (&A)
   }
 }
 
+// Operands of block W0 + wb (wb a runtime value in 0..3, resolved by an unrolled switch).
+template <int R, int W0>
+__device__ __forceinline__ void build_slice_operands(const LaneWords& L, int wb, uint32_t (&A)[2][4]) {
+  switch (wb) {
+    case 0: build_operands<R, W0>(L, A); break;
+    case 1: if constexpr (W0 + 1 < 8) build_operands<R, W0 + 1>(L, A); break;
+    case 2: if constexpr (W0 + 2 < 8) build_operands<R, W0 + 2>(L, A); break;
+    default: if constexpr (W0 + 3 < 8) build_operands<R, W0 + 3>(L, A); break;
+  }
+}
+
 }  // namespace matq

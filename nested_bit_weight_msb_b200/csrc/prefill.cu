@@ -23,13 +23,14 @@
 // for |x| in the fp16 normal range).
 //
 // Every mbarrier wait is bounded (about a second of clock); on expiry the kernel records an
-// error code in the workspace flag, every role drains, TMEM is freed, and the kernel returns.
+// error code in the workspace header, every role drains, TMEM is freed, and the kernel returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
 #include "operands.cuh"
+#include "sync.cuh"
 
 namespace matq {
 
@@ -40,100 +41,11 @@ constexpr int kAStages = 3;     // fp16 weight-tile ring
 constexpr int kBStages = 3;     // activation-tile ring
 constexpr int kThreads = 256;
 constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
-
-// ---- PTX wrappers --------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false (and the error flag set) if the phase did not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
-      atomicOr(err, code);
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(smem_u32(dst)),
-      "l"((uint64_t)map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// SW128 K-major shared-memory matrix descriptor (rows of 128 bytes, 8-row groups 1024 B apart).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                           uint32_t accum) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-      : "memory");
-}
-
-__device__ __forceinline__ void stmatrix_x4(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-  asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(r0), "r"(r1),
-               "r"(r2), "r"(r3)
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // ---- activation conversion -----------------------------------------------------------------
-__global__ void xprep_prefill_kernel(const uint16_t* __restrict__ x, size_t n, __half* __restrict__ x16,
-                                     int* __restrict__ err) {
-  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
+__global__ void xprep_prefill_kernel(const uint16_t* __restrict__ x, size_t n, __half* __restrict__ x16) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t nvec = n / 8;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
@@ -237,7 +149,7 @@ __device__ __forceinline__ void dequant_block(const LaneWords& L, const __half2 
       const int rsel = rho & 1;  // rho 0, 2: row gid; rho 1, 3: row gid + 8
       __half2 u;
       if constexpr (R == 8) {
-        u = __hsub2(v, __hadd2(k1024, dz2[rsel]));  // dz2 holds -z here: v - 1024 - z, exact
+        u = __hsub2(v, __hadd2(k1024, dz2[rsel]));  // dz2 holds z here: v - (1024 + z), exact
       } else {
         u = __hfma2(__hsub2(v, k1024), __float2half2_rn(code_mult<R>(rho)), dz2[rsel]);
       }
@@ -324,6 +236,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  pdl_launch_dependents();
+  pdl_wait();  // x16 comes from the conversion kernel; y may be read by earlier kernels
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -432,10 +346,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
 }
 
 // ---- host side -----------------------------------------------------------------------------
-size_t prefill_workspace_bytes(int M, int K, int group) {
-  (void)group;
-  return ((((size_t)M * K * 2) + 255) & ~size_t(255)) + 256;
-}
+size_t prefill_scratch_bytes(int M, int K) { return (((size_t)M * K * 2) + 255) & ~size_t(255); }
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -468,8 +379,8 @@ static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
   if (e != cudaSuccess) return e;
   dim3 grid((P.N + kBM - 1) / kBM, (P.M + BN - 1) / BN);
-  kern<<<grid, kThreads, S::kTotal, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], P);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3], maps[4],
+                    maps[5], P);
 }
 
 template <int BN, int GROUP>
@@ -487,16 +398,14 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
                            const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
                            cudaStream_t s) {
   uint8_t* ws = (uint8_t*)workspace;
-  const size_t x16_bytes = (((size_t)M * K * 2) + 255) & ~size_t(255);
-  __half* x16 = (__half*)ws;
-  int* err = (int*)(ws + x16_bytes);
+  int* err = (int*)(ws + 4);  // sticky prefill error word in the workspace header
+  __half* x16 = (__half*)(ws + workspace_header_bytes());
   {
     const size_t n = (size_t)M * K;
     int blocks = (int)((n / 8 + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks < 1) blocks = 1;
-    xprep_prefill_kernel<<<blocks, 256, 0, s>>>((const uint16_t*)x, n, x16, err);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(xprep_prefill_kernel, dim3(blocks), dim3(256), 0, s, (const uint16_t*)x, n, x16);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap maps[6];

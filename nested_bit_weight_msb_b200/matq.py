@@ -54,6 +54,8 @@ _SIGNATURES = {
     "matq_slice": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_int, _c_vp, _c_vp]),
     "matq_slice_copy": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_int, _c_vp, _c_size, _c_vp]),
     "matq_linear_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "matq_workspace_init": (_c_int, [_c_vp, _c_size, _c_vp]),
+    "matq_workspace_status": (_c_int, [_c_vp, ctypes.POINTER(_c_int)]),
     "matq_linear": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
     "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
@@ -136,6 +138,19 @@ def workspace_bytes(M: int, K: int, N: int, group: int) -> int:
     return int(matq_linear_workspace(M, K, N, group))
 
 
+def workspace(M: int, K: int, N: int, group: int, device="cuda"):
+    """A zero-filled workspace (uint8 CUDA tensor) for calls up to these sizes."""
+    torch = _torch()
+    return torch.zeros(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=device)
+
+
+def workspace_status(ws) -> int:
+    """Device status word of a workspace (0 = every call so far completed normally)."""
+    out = _c_int(0)
+    check(matq_workspace_status(_ptr(ws), ctypes.byref(out)), "matq_workspace_status")
+    return int(out.value)
+
+
 def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=None,
            y_mode: int = MATQ_OUT_BF16, workspace=None, stream=None):
     """y = x . W_hat_r^T.  x: [M, K] bf16 CUDA tensor; scales: [N, K/group] (fp16 or int16
@@ -146,7 +161,7 @@ def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=
         dt = torch.bfloat16 if y_mode == MATQ_OUT_BF16 else torch.float32
         y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, N), dtype=dt, device=x.device)
     if workspace is None:
-        workspace = torch.empty(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
     check(matq_linear(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
                       _ptr(y), y_mode, _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "matq_linear")
     return y

@@ -105,6 +105,14 @@ def test_linear_rejects(M):
     assert call(ws_bytes=16) == M.MATQ_ESIZE
 
 
+def test_workspace_init_rejects(M):
+    assert M.matq_workspace_init(None, 1 << 20, None) == M.MATQ_ENULL
+    assert M.matq_workspace_init(FAKE + 4, 1 << 20, None) == M.MATQ_EALIGN
+    assert M.matq_workspace_init(FAKE, 16, None) == M.MATQ_ESIZE
+    import ctypes
+    assert M.matq_workspace_status(None, ctypes.byref(ctypes.c_int(0))) == M.MATQ_ENULL
+
+
 def test_glue_rejects(M):
     assert M.matq_rmsnorm(FAKE, 0, 16, 1e-5, FAKE, None) == M.MATQ_EINVAL_SHAPE
     assert M.matq_rmsnorm(None, 1, 16, 1e-5, FAKE, None) == M.MATQ_ENULL
