@@ -48,12 +48,17 @@ METRIC = "sliced r-bit linear: decode weight GB/s vs HBM peak; prefill TFLOP/s p
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
     ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["decode", "prefill"], default=None,
+                    help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
+    ap.add_argument("--r", type=int, default=2)
+    ap.add_argument("--m", type=int, default=1)
+    ap.add_argument("--calls", type=int, default=8)
     return ap.parse_args()
 
 
@@ -130,7 +135,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         return self
@@ -348,7 +353,9 @@ def run_ours(args):
                        "parallelism": f"replicas x{world}", "timing": "CUDA graph replay, CUDA events"},
             "roofline": rl,
             "e2e": e2e,
-            "gpu_launches": args.steps * len(calls) * (3 * 2 + 1),
+            # per FFN: gate, up, down (one kernel each on the decode path, conversion + GEMM on
+            # the prefill path) and the SiLU-gated product
+            "gpu_launches": args.steps * len(calls) * (3 * (1 if spec["unit"] == "GB/s" else 2) + 1),
             "clocks": clk.summary(),
             "peaks_source": peaks.get("_source"),
         }
@@ -441,8 +448,33 @@ def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
             "ms_per_step": ms}
 
 
+def run_case(args):
+    """A few single calls of the gate projection (14336 x 4096, group 128) at width r and
+    batch m, rotating through device copies of the pack (> L2); used for ncu captures."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq, synth
+    torch.cuda.set_device(0)
+    q, s, z = synth.parent_weights(D_FF, D_MODEL, GROUP, seed=0, proj="gate")
+    p0 = matq.pack(torch.from_numpy(q).cuda(), r_keep=8)
+    packs = [p0] + [p0.clone() for _ in range(args.copies - 1)]
+    ds = torch.from_numpy(s.view(np.int16)).cuda()
+    dz = torch.from_numpy(z).cuda()
+    xb, _ = synth.activations(args.m, D_MODEL, seed=0, outlier_frac=0.01 if args.case == "prefill" else 0.0)
+    dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    ws = matq.workspace(args.m, D_MODEL, D_FF, GROUP)
+    y = torch.empty((args.m, D_FF), dtype=torch.bfloat16, device="cuda")
+    for i in range(args.calls):
+        matq.linear(dx, packs[i % len(packs)], 8, ds, dz, D_FF, args.r, GROUP, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    assert matq.workspace_status(ws) == 0
+    print(json.dumps({"case": args.case, "r": args.r, "m": args.m, "calls": args.calls, "ok": True}))
+    return 0
+
+
 def main():
     args = parse()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

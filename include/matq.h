@@ -137,7 +137,8 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r,
  * (matq_workspace_init, or any zero fill); every successful call leaves it zero again, so a
  * workspace is reused without re-initialisation.  Calls that share a workspace must be
  * ordered on the device (one stream, or synchronised streams).  A workspace sized for
- * (M_max, K_max, N) serves every call with M <= M_max and K <= K_max on either path. */
+ * (M_max, K_max, N) serves every call with M <= M_max and K <= K_max on either path
+ * (a decode-sized one serves prefill only for M <= 16). */
 size_t matq_linear_workspace(int M, int K, int N, int group);
 
 /* Zero the workspace header (asynchronous on `stream`).  ws_bytes: capacity of workspace. */

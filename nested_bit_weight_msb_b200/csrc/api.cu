@@ -117,7 +117,11 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r, void* p
 
 size_t matq_linear_workspace(int M, int K, int N, int group) {
   if (M < 1 || N < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
-  return M <= kDecodeMaxM ? decode_workspace_bytes(M) : workspace_header_bytes() + prefill_scratch_bytes(M, K);
+  // sized so that it also serves every smaller M (decode or prefill) with these K, N
+  const size_t dec = decode_workspace_bytes(M <= kDecodeMaxM ? M : kDecodeMaxM);
+  if (M <= kDecodeMaxM) return dec;
+  const size_t pre = workspace_header_bytes() + prefill_scratch_bytes(M, K);
+  return pre > dec ? pre : dec;
 }
 
 int matq_workspace_init(void* workspace, size_t ws_bytes, void* stream) {

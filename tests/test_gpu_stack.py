@@ -1,0 +1,91 @@
+"""GPU parity of the Mix'n'Match stack glue and of a small mixed-width FFN stack.
+
+Each step is checked teacher-forced: the oracle gets the GPU's own input for that step
+(RMSNorm of the GPU's residual stream, the projections of the GPU's normalised input, the
+gated product of the GPU's gate/up outputs, the down projection of the GPU's product), at the
+stated tolerance.  The end-to-end deviation of the whole stack from an fp64 run of the oracle
+alone is reported (and only checked to be finite and small in a loose sense).
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from helpers import check_close
+from nested_bit_weight_msb_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def M():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from nested_bit_weight_msb_b200 import matq
+    return matq
+
+
+def _bf16(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("Mt,D", [(1, 4096), (16, 4096), (33, 1000)])
+def test_rmsnorm(M, Mt, D):
+    import torch
+    rng = np.random.default_rng(D + Mt)
+    h = (rng.standard_normal((Mt, D)) * rng.uniform(0.1, 30)).astype(np.float32)
+    n = M.rmsnorm(torch.from_numpy(h).cuda(), eps=1e-5)
+    check_close(_bf16(n), O.rmsnorm(h, 1e-5), what="rmsnorm")
+
+
+@pytest.mark.parametrize("Mt,F", [(1, 14336), (16, 14336), (3, 1001)])
+def test_silu_mul(M, Mt, F):
+    import torch
+    rng = np.random.default_rng(F + Mt)
+    gb, gv = synth.bf16_round((rng.standard_normal((Mt, F)) * 3).astype(np.float32))
+    ub, uv = synth.bf16_round(rng.standard_normal((Mt, F)).astype(np.float32))
+    g = torch.from_numpy(gb.view(np.int16)).cuda().view(torch.bfloat16)
+    u = torch.from_numpy(ub.view(np.int16)).cuda().view(torch.bfloat16)
+    a = M.silu_mul(g, u)
+    check_close(_bf16(a), O.gated_product(gv, uv), what="silu_mul")
+
+
+@pytest.mark.parametrize("Mt", [1, 16, 40])
+def test_mixnmatch_stack_teacher_forced(M, Mt):
+    import torch
+    D, F, G, L = 512, 1024, 128, 4
+    widths = [2, 4, 3, 8]
+    layers = []
+    for l in range(L):
+        lay = {}
+        for name, (N, K) in (("gate", (F, D)), ("up", (F, D)), ("down", (D, F))):
+            q, s, z = synth.parent_weights(N, K, G, seed=3, layer=l, proj=name)
+            dq = torch.from_numpy(q).cuda()
+            lay[name] = dict(host=(q, s, z), planes=M.pack(dq, r_keep=widths[l]),
+                             s=torch.from_numpy(s.view(np.int16)).cuda(), z=torch.from_numpy(z).cuda(), N=N)
+        layers.append(lay)
+    xb, xv = synth.activations(Mt, D, seed=5)
+    h = torch.from_numpy(xv.copy()).cuda()           # fp32 residual stream
+    ws = M.workspace(Mt, F, F, G)
+    h_ref = xv.astype(np.float64)                     # oracle-only run, for the reported deviation
+    for l, lay in enumerate(layers):
+        r = widths[l]
+        n = M.rmsnorm(h, eps=1e-5)
+        check_close(_bf16(n), O.rmsnorm(h.cpu().numpy(), 1e-5), what=f"layer {l} rmsnorm")
+        outs = {}
+        for name in ("gate", "up"):
+            p = lay[name]
+            outs[name] = M.linear(n, p["planes"], r, p["s"], p["z"], p["N"], r, G, workspace=ws)
+            check_close(_bf16(outs[name]), O.linear(_bf16(n), *p["host"], r, G), what=f"layer {l} {name}")
+        a = M.silu_mul(outs["gate"], outs["up"])
+        check_close(_bf16(a), O.gated_product(_bf16(outs["gate"]), _bf16(outs["up"])), what=f"layer {l} silu")
+        h_before = h.cpu().numpy().astype(np.float64)
+        p = lay["down"]
+        M.linear(a, p["planes"], r, p["s"], p["z"], p["N"], r, G, y=h, y_mode=M.MATQ_OUT_F32_ACCUM, workspace=ws)
+        check_close(h.cpu().numpy() - h_before, O.linear(_bf16(a), *p["host"], r, G), what=f"layer {l} down")
+        h_ref = O.ffn_block(h_ref, {k: v["host"] for k, v in lay.items()}, r, G)
+    assert M.workspace_status(ws) == 0
+    dev = np.linalg.norm(h.cpu().numpy() - h_ref) / np.linalg.norm(h_ref)
+    print(f"end-to-end stack deviation (M={Mt}): {dev:.3e}")
+    assert np.isfinite(dev) and dev < 5e-2
