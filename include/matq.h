@@ -81,6 +81,7 @@ extern "C" {
 #define MATQ_ESIZE         -8   /* a caller buffer (planes, workspace) is too small          */
 #define MATQ_EDTYPE        -9   /* unknown output mode                                      */
 #define MATQ_EDEVICE      -10   /* current device is not sm_100 (B200 class)               */
+#define MATQ_ESCRATCH     -11   /* sizes exceed matq_linear_noalloc's fixed scratch        */
 
 /* ---- output modes of matq_linear ----------------------------------------------------- */
 #define MATQ_OUT_BF16       0   /* y [M, N] bf16 = x . W_hat^T                             */
@@ -170,6 +171,52 @@ int matq_linear(const void* x, int M, int K,
                 int r, int group,
                 void* y, int y_mode,
                 void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- the sliced linear layer without a caller workspace -------------------------------- */
+
+/* Capacity, in bytes, of the scratch array that libmatq itself holds for matq_linear_noalloc
+ * (one array per device, in static device memory). */
+#define MATQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* matq_linear with the scratch held by libmatq instead of a caller workspace.  This entry
+ * point is a library convenience; the sliced-quantisation papers have no counterpart of it.
+ *
+ * Who needs it: callers that must not allocate device memory at call time and have none to
+ * spare for a workspace: a host runtime or plugin that owns every allocation itself and
+ * hands the library only its tensors; serving loops where cudaMalloc/cudaFree (which may
+ * synchronise the device, and may fail once memory is fragmented) are banned on the hot
+ * path; C callers without a memory allocator of their own.  The call allocates nothing on
+ * the device or the host, through CUDA or any other library; its scratch is a fixed
+ * MATQ_NOALLOC_SCRATCH_BYTES array in libmatq's static device memory.
+ *
+ * Arguments, output and kernels are those of matq_linear (same results), except:
+ *   status_out  optional (NULL: not reported) device pointer to one int, 4-byte aligned.
+ *               After the call completes on the device it holds 0, or the device-side
+ *               wait-timeout code of this call (then y is undefined).
+ *   no workspace arguments.
+ * Limits: the sizes must fit the fixed scratch, i.e. matq_linear_workspace(M, K, N, group)
+ * <= MATQ_NOALLOC_SCRATCH_BYTES; larger calls return MATQ_ESCRATCH and launch nothing.
+ * Every M <= 16 (decode path) fits; M > 16 (prefill path) fits while 262,400 + M*K*2 bytes
+ * (rounded up to 256) do, e.g. M <= 991 at K = 4096.  Use matq_linear with a caller workspace beyond that.
+ * Set-up: the first call on each device, made with that device current, looks up the device
+ * address of the array (cudaGetSymbolAddress; this can load libmatq's device code onto the
+ * device) and caches it; a failure returns MATQ_ECUDA.  Make that first call before any
+ * stream capture is started on the device.
+ * State: unlike the other entry points, this one keeps state between calls: the array and
+ * its cached address.
+ * Sharing: every call on a device uses the same array, which keeps its last contents; each
+ * call first clears the part that must start at zero (an asynchronous memset of the header
+ * on `stream`), then launches the kernel, then copies the status word (if status_out).
+ * Calls whose executions overlap on the device (different streams, not ordered with one
+ * another, or different host threads with such streams) race on the array and give wrong
+ * results: order them (one stream, or events).  A cudaDeviceReset invalidates the cached
+ * address; do not call this entry point on that device afterwards in the same process. */
+int matq_linear_noalloc(const void* x, int M, int K,
+                        const void* planes, int r_keep,
+                        const uint16_t* scales, const uint8_t* zeros, int N,
+                        int r, int group,
+                        void* y, int y_mode,
+                        int* status_out, void* stream);
 
 /* ---- glue of the Mix'n'Match FFN stack ------------------------------------------------- */
 

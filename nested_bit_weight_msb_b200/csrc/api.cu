@@ -49,6 +49,12 @@ size_t packed_bytes(int N, int K, int r_keep) {
 
 }  // namespace
 
+namespace matq {
+// Status helpers for the other translation units of the C ABI.
+int record_cuda_error(cudaError_t e) { return cuda_status(e); }
+int check_sm100_device() { return check_device(); }
+}  // namespace matq
+
 extern "C" {
 
 int matq_version(void) { return 100; }
@@ -66,6 +72,9 @@ const char* matq_strerror(int status) {
     case MATQ_ESIZE: return "caller buffer too small";
     case MATQ_EDTYPE: return "unknown output mode";
     case MATQ_EDEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    case MATQ_ESCRATCH:
+      return "sizes need more scratch than matq_linear_noalloc's fixed array (MATQ_NOALLOC_SCRATCH_BYTES); "
+             "use matq_linear with a caller workspace";
     default: return "unknown status";
   }
 }

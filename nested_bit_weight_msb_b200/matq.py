@@ -35,6 +35,7 @@ MATQ_ECUDA = -7
 MATQ_ESIZE = -8
 MATQ_EDTYPE = -9
 MATQ_EDEVICE = -10
+MATQ_ESCRATCH = -11
 MATQ_OUT_BF16 = 0
 MATQ_OUT_F32 = 1
 MATQ_OUT_F32_ACCUM = 2
@@ -58,6 +59,8 @@ _SIGNATURES = {
     "matq_workspace_status": (_c_int, [_c_vp, ctypes.POINTER(_c_int)]),
     "matq_linear": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
+    "matq_linear_noalloc": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
+                                     _c_vp, _c_int, _c_vp, _c_vp]),
     "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
     "matq_silu_mul": (_c_int, [_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_vp]),
 }
@@ -164,6 +167,22 @@ def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=
         workspace = torch.zeros(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
     check(matq_linear(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
                       _ptr(y), y_mode, _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "matq_linear")
+    return y
+
+
+def linear_noalloc(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=None,
+                   y_mode: int = MATQ_OUT_BF16, status=None, stream=None):
+    """Same as ``linear`` but with libmatq's own fixed scratch (no workspace argument).
+    ``status``: optional int32 CUDA tensor of one element that receives the call's device
+    status word.  Returns y."""
+    torch = _torch()
+    M, K = x.shape
+    if y is None:
+        dt = torch.bfloat16 if y_mode == MATQ_OUT_BF16 else torch.float32
+        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, N), dtype=dt, device=x.device)
+    sp = _ptr(status) if status is not None else None
+    check(matq_linear_noalloc(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
+                              _ptr(y), y_mode, sp, _stream_ptr(stream)), "matq_linear_noalloc")
     return y
 
 
