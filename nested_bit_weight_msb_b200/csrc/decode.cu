@@ -184,10 +184,11 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
       for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
 
   bool ok = true;
+  // (row group, chunk) of the current item, advanced item by item (no division in the loop)
+  const int rg_first = (int)(ib / P.KC);
+  int rg = rg_first, kc = (int)(ib - (long long)rg_first * P.KC);
   for (int n = 0; n < nitems; ++n) {
     const int s = n % kDecStages;
-    const long long it = ib + n;
-    const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
     if (ok) ok = mbar_wait(&full[s], (n / kDecStages) & 1, P.err, 2);
     if (ok) {
       const uint8_t* st = smem + s * Lt::kStage;
@@ -219,7 +220,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
             float sv = 0.f, zv = 0.f;
             if (row < P.N) {
               sv = __half2float(*reinterpret_cast<const __half*>(st + Lt::oS + rr * 8 + gl * 2));
-              const int zoff = (int)(((size_t)row * P.G + (size_t)kc * NG) & 3);
+              const int zoff = (int)(((unsigned)row * (unsigned)P.G + (unsigned)kc * NG) & 3u);
               zv = (float)st[Lt::oZ + rr * 4 + zoff + gl];
             }
             a[h] = sv * amul[h];
@@ -267,12 +268,19 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
     // the streaming warps (0..7) refill this slot with item n + S once every warp released it
     if (rs + kRowSlices * KS < 8 && n + kDecStages < nitems && ok) {
       ok = mbar_wait(&empty[s], (n / kDecStages) & 1, P.err, 1);
-      if (ok) refill(n + kDecStages);
+      if (ok) {
+        int rg2 = rg, kc2 = kc + kDecStages;
+        while (kc2 >= P.KC) {
+          kc2 -= P.KC;
+          ++rg2;
+        }
+        refill(n + kDecStages, rg2, kc2);
+      }
     }
 
     // flush at the end of a row group (or of this CTA's range); all warps get here for the
     // same items, so the four k-slices of a row slice meet at a named barrier
-    if (n == nitems - 1 || (it + 1) / P.KC != rg) {
+    if (n == nitems - 1 || kc == P.KC - 1) {
       const long long g0 = (long long)rg * P.KC, g1 = g0 + P.KC;
       const bool whole = g0 >= ib && g1 <= ie;
       if (KS > 0) {
@@ -324,7 +332,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
           const long long cf = item_owner(g0, P.I, P.C), cl = item_owner(g1 - 1, P.I, P.C);
           int* cnt = &P.counters[rg * kRowSlices + rs];
           if (c != cf) {
-            const int side = (rg == (int)(ib / P.KC)) ? 0 : 1;
+            const int side = (rg == rg_first) ? 0 : 1;
             float4* mine = reinterpret_cast<float4*>(
                 P.partial + ((size_t)(c * 2 + side) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
@@ -405,6 +413,10 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
 #pragma unroll
           for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
     }
+    if (++kc == P.KC) {
+      kc = 0;
+      ++rg;
+    }
   }
 }
 
@@ -447,11 +459,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   pdl_launch_dependents();
 
   // Planes of item n into slot n % S (2-D TMA by thread 0): they depend on no earlier kernel.
-  auto stream_planes = [&](int n) {
+  auto stream_planes = [&](int n, int rg, int kc) {
     if (threadIdx.x == 0) {
       const int s = n % kDecStages;
-      const long long it = ib + n;
-      const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
       uint8_t* st = smem + s * Lt::kStage;
       mbar_expect_tx_only(&full[s], Lt::kPlanes + mrows * kChunk * 2);
 #pragma unroll
@@ -461,10 +471,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   };
   // Activation rows (a bulk copy per token), scales and zero points (cp.async, one row per
   // streamer thread) of item n; called by the streamer threads (warps 0..7) only.
-  auto stream_rest = [&](int n) {
+  auto stream_rest = [&](int n, int rg, int kc) {
     const int s = n % kDecStages;
-    const long long it = ib + n;
-    const int rg = (int)(it / P.KC), kc = (int)(it % P.KC);
     uint8_t* st = smem + s * Lt::kStage;
     const int t = threadIdx.x;
     if (t < mrows) bulk_load(st + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk, kChunk * 2, &full[s]);
@@ -493,16 +501,23 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     }
     if (t == 0) mbar_arrive(&full[s]);
   };
-  auto refill = [&](int n) {
-    stream_planes(n);
-    stream_rest(n);
+  auto refill = [&](int n, int rg, int kc) {
+    stream_planes(n, rg, kc);
+    stream_rest(n, rg, kc);
   };
 
   const int pre = nitems < kDecStages ? nitems : kDecStages;
-  for (int n = 0; n < pre; ++n) stream_planes(n);
+  const int rg0 = (int)(ib / P.KC), kc0 = (int)(ib - (long long)rg0 * P.KC);
+  for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
+    stream_planes(n, rg, kc);
+    if (++kc == P.KC) { kc = 0; ++rg; }
+  }
   pdl_wait();  // activations, counters and y belong to earlier kernels in the stream
   if (warp < 8)
-    for (int n = 0; n < pre; ++n) stream_rest(n);
+    for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
+      stream_rest(n, rg, kc);
+      if (++kc == P.KC) { kc = 0; ++rg; }
+    }
 
   const int rs = warp & 3, ks = warp >> 2;
   if constexpr (Lt::KSL == 2) {
