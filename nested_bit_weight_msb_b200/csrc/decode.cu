@@ -11,10 +11,10 @@
 // against the fp16 bit pattern of 1024 gives 1024 + sigma * v exactly (operands.cuh).  The
 // per-register powers of two sigma split into a per-row factor alpha (folded into the group
 // scale) and a per-input factor beta (inputs 8..15 of every 16-input MMA slice enter the B
-// operand divided by 16 for r <= 4, exact in fp16).  Two more MMAs per 16-input slice, with
-// constant A operands, accumulate the per-token sums the algebra needs in registers:
-// Dc = sum_k (-1024) * B_k (removes the 1024 bias) and Ds = sum_k beta_k * B_k = sum_k x_k
-// (the zero-point term).  Per 64-input slice of a group, in fp32:
+// operand divided by 16 for r <= 4, exact in fp16).  One more MMA per 16-input slice, with a
+// constant A operand (rows 0..7: -1024, rows 8..15: beta_k), accumulates both per-token sums
+// the algebra needs in registers: Dc = sum_k (-1024) * B_k (removes the 1024 bias) and
+// Ds = sum_k beta_k * B_k = sum_k x_k (the zero-point term).  Per slice of a group, in fp32:
 //
 //   y += a_row * (D + Dc) + s * (delta_r - z) * Ds,   a_row = s * 2^(8-r) / alpha_row
 //
@@ -26,8 +26,8 @@
 // (stream-K style) and streams each into a shared-memory ring: the planes of width r (one
 // 2-D TMA per plane: exactly r bits per weight leave HBM), the chunk's bf16 activation rows
 // (one bulk copy per token into padded rows, so fragment loads are conflict-free) and the
-// rows' scales and zero points (cp.async).  Sixteen warps split each item 4 x 4: four row
-// slices of RPW row tiles times four 64-input slices; each warp reuses every activation
+// rows' scales and zero points (cp.async).  Eight warps split each item 4 x 2: four row
+// slices of RPW row tiles times two 128-input slices; each warp reuses every activation
 // fragment across its row tiles.  Row groups inside a CTA's range are written directly.  A
 // row group split between CTAs is combined deterministically by its first contributor,
 // which works on it last: the others store their partial sums in their workspace slots and
@@ -172,8 +172,10 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   else if constexpr (R == 3) { amul[0] = amul[1] = 32.f; }
   else if constexpr (R == 4) { amul[0] = amul[1] = 16.f; }
   else { amul[0] = amul[1] = 1.f; }
-  const uint32_t Ac[4] = {kNeg1024, kNeg1024, kNeg1024, kNeg1024};
-  const uint32_t As[4] = {kOne, kOne, kBetaHi, kBetaHi};
+  // One constant-A MMA yields both token sums: A rows 0..7 are -1024 (D rows 0..7 = Dc) and
+  // rows 8..15 are beta_k (D rows 8..15 = Ds).  Fragment registers: {row g, k lo}, {row g+8,
+  // k lo}, {row g, k hi}, {row g+8, k hi}; result {Dc(t), Dc(t+1), Ds(t), Ds(t+1)}.
+  const uint32_t Acs[4] = {kNeg1024, kOne, kNeg1024, kBetaHi};
 
   float yacc[RPW][NT][4];
 #pragma unroll
@@ -196,33 +198,34 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
 #pragma unroll
       for (int j = 0; j < RPW; ++j) lds_slice_words<R, RG, NB, KS>(st, rs * RPW + j, lane, L[j]);
 
-      float d[RPW][NT][4], dc[NT][4], ds[NT][4];
+      float d[RPW][NT][4], dcs[NT][4];
       auto zero_acc = [&]() {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            dc[nt][i] = 0.f;
-            ds[nt][i] = 0.f;
+            dcs[nt][i] = 0.f;
 #pragma unroll
             for (int j = 0; j < RPW; ++j) d[j][nt][i] = 0.f;
           }
       };
-      // fold the inputs accumulated so far (all in scale group gl) into the running sums
+      // Byte offset of this lane's zero points inside their 4-byte windows: the same for every
+      // row the lane touches in the item (the rows differ by multiples of 8, and 8 * G is a
+      // multiple of 4).
+      const int zoff = (int)(((unsigned)gid * (unsigned)P.G + (unsigned)kc * NG) & 3u);
+      const uint8_t* srow = st + Lt::oS + (rs * RPW * 16 + gid) * 8;
+      const uint8_t* zrow = st + Lt::oZ + (rs * RPW * 16 + gid) * 4 + zoff;
+      // fold the inputs accumulated so far (all in scale group gl) into the running sums.
+      // Rows >= N read stale scales and zero points; their sums are never stored.
       auto promote = [&](int gl) {
 #pragma unroll
         for (int j = 0; j < RPW; ++j) {
           float a[2], cz[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int rr = (rs * RPW + j) * 16 + gid + 8 * h;  // row inside the item
-            const int row = rg * RG * 16 + rr;
-            float sv = 0.f, zv = 0.f;
-            if (row < P.N) {
-              sv = __half2float(*reinterpret_cast<const __half*>(st + Lt::oS + rr * 8 + gl * 2));
-              const int zoff = (int)(((unsigned)row * (unsigned)P.G + (unsigned)kc * NG) & 3u);
-              zv = (float)st[Lt::oZ + rr * 4 + zoff + gl];
-            }
+            const int rr = j * 16 + 8 * h;  // row offset inside the warp's row slice
+            const float sv = __half2float(*reinterpret_cast<const __half*>(srow + rr * 8 + gl * 2));
+            const float zv = (float)zrow[rr * 4 + gl];
             a[h] = sv * amul[h];
             cz[h] = sv * (kDelta - zv);
           }
@@ -230,7 +233,8 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              yacc[j][nt][i] = fmaf(cz[i >> 1], ds[nt][i], fmaf(a[i >> 1], d[j][nt][i] + dc[nt][i], yacc[j][nt][i]));
+              yacc[j][nt][i] = fmaf(cz[i >> 1], dcs[nt][2 + (i & 1)],
+                                    fmaf(a[i >> 1], d[j][nt][i] + dcs[nt][i & 1], yacc[j][nt][i]));
         }
         zero_acc();
       };
@@ -248,8 +252,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
         for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            mma_f16(dc[nt], Ac, b0[jj][nt], b1[jj][nt]);
-            mma_f16(ds[nt], As, b0[jj][nt], b1[jj][nt]);
+            mma_f16(dcs[nt], Acs, b0[jj][nt], b1[jj][nt]);
           }
 #pragma unroll
         for (int j = 0; j < RPW; ++j) {
