@@ -118,6 +118,14 @@ def max_over_ranks(world, value, device):
     return float(t.item())
 
 
+def whole_job_value(unit, step_bytes, step_flops, world, ms_step):
+    """Whole-job throughput: every rank runs the same step on its own batches (weak scaling),
+    so the job moves world x the per-rank units in the slowest rank's step time."""
+    if unit == "GB/s":
+        return step_bytes * world / (ms_step * 1e-3) / 1e9
+    return step_flops * world / (ms_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------------------------------
 # clocks
 # ---------------------------------------------------------------------------------------------
@@ -177,11 +185,11 @@ class ClockSampler:
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------
 
-def cpu_oracle_rate(spec, weights_host, budget_s=12.0):
-    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: rows of
-    the three FFN matrices at each (r, M), scaled to the metric's unit per second."""
+def cpu_oracle_rate(spec, weights_host, budget_s=12.0, rows=256):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: the first
+    `rows` rows of the three FFN matrices at each (r, M), scaled to the metric's unit per
+    second.  At least one pass over every (r, M) is made."""
     import oracle as O
-    rows = 256
     done_b = done_f = 0.0
     t0 = time.perf_counter()
     rng = np.random.default_rng(0)
@@ -229,11 +237,14 @@ def run_reference(args):
         return 0
     spec = workload_spec(args.workload)
     w = host_weights()
+    # each step is a bounded sample, sized so that warm-up + steps stay within ~3 minutes
+    budget = min(5.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = 256 if budget >= 2.0 else 32
     for _ in range(args.warmup):
-        cpu_oracle_rate(spec, w, budget_s=0.5)
+        cpu_oracle_rate(spec, w, budget_s=budget, rows=rows)
     vals = []
     for _ in range(args.steps):
-        vals.append(cpu_oracle_rate(spec, w, budget_s=5.0))
+        vals.append(cpu_oracle_rate(spec, w, budget_s=budget, rows=rows))
     v = float(np.mean([c["value"] for c in vals]))
     b, f = step_units(spec)
     per_step_units = b / 1e9 if spec["unit"] == "GB/s" else f / 1e12
@@ -329,10 +340,7 @@ def run_ours(args):
     ms_total = max_over_ranks(world, e0.elapsed_time(e1), dev)
     ms_step = ms_total / args.steps
     b, f = step_units(spec)
-    if spec["unit"] == "GB/s":
-        value = b * world / (ms_step * 1e-3) / 1e9
-    else:
-        value = f * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(spec["unit"], b, f, world, ms_step)
 
     # ---- roofline of the dominant kernel: per-call device time of the sliced linear ----------
     rl = roofline(args, spec, linear, xs, gate_buf, stream, dev)
@@ -359,7 +367,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "peaks_source": peaks.get("_source"),
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_oracle_rate(spec, weights)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -379,38 +387,80 @@ def load_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "_source": "fallback"}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the roofline
+# kernel, from an ncu capture, with the SHA-256 of the kernel's sources at capture time; the
+# figure is reported only while the sources are unchanged.  Captures: profiles/.
+_KERNEL_SOURCES = {
+    "decode": ("decode.cu", "common.cuh", "operands.cuh", "sync.cuh"),
+    "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
+}
+NCU_TRAFFIC = {
+    "decode": {"sha256": None, "bytes": None},
+    "prefill": {"sha256": "a5e3008895282b04070e43528239556d29fe4623998745f67f56acc196650174", "bytes": 51_869_952 + 31_986_432},
+}
+
+
+def kernel_source_sha(path_kind):
+    import hashlib
+    h = hashlib.sha256()
+    for f in _KERNEL_SOURCES[path_kind]:
+        with open(os.path.join(ROOT, "nested_bit_weight_msb_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(path_kind):
+    rec = NCU_TRAFFIC[path_kind]
+    if rec["bytes"] is None or rec["sha256"] != kernel_source_sha(path_kind):
+        return None
+    return rec["bytes"]
+
+
 def roofline(args, spec, linear, xs, gate_buf, stream, dev):
-    """Average device duration of single sliced-linear calls (the dominant kernel and its
-    activation pre-pass), measured with CUDA events on the launching stream while a
-    preceding spin kernel keeps the host ahead of the device."""
+    """Average device time per launch of the dominant kernel in steady state: a CUDA graph of
+    back-to-back sliced-linear calls on the gate matrix (rotating weight copies, so every call
+    streams from HBM), timed with CUDA events on the launching stream; total / launches."""
     import torch
     peaks = load_peaks()
     M = max(spec["batches"]) if spec["unit"] == "TFLOP/s" else 1
     r = 2 if spec["unit"] == "GB/s" else 4
     n = 24
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
     with torch.cuda.stream(stream):
-        torch.cuda._sleep(int(2e8))
-        for i in range(n):
-            ev[i].record(stream)
+        for i in range(3):
             linear("gate", i % args.copies, xs[M], r, gate_buf[M])
-        ev[n].record(stream)
         torch.cuda.synchronize()
-    durs = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
-    avg_ms = float(np.mean(durs[2:]))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                linear("gate", i % args.copies, xs[M], r, gate_buf[M])
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = []
+        for _ in range(5):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            reps.append(e0.elapsed_time(e1) / n)
+    del g
+    avg_ms = float(np.median(reps))
     if spec["unit"] == "GB/s":
         units = linear_bytes(M, D_FF, D_MODEL, r)
         ach = units / (avg_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": None, "kernel": f"matq_linear decode (gate 14336x4096, r={r}, M={M}), per call",
-                "avg_us": avg_ms * 1e3, "peak_source": peaks.get("_source")}
+                "traffic": measured_traffic("decode"), "algorithmic_bytes": units,
+                "kernel": f"decode_kernel via matq_linear (gate 14336x4096, r={r}, M={M})",
+                "avg_us": avg_ms * 1e3, "launches_timed": n, "peak_source": peaks.get("_source")}
     flops = 2 * M * D_FF * D_MODEL
     ach = flops / (avg_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-            "traffic": None, "kernel": f"matq_linear prefill (gate 14336x4096, r={r}, M={M}), per call",
-            "avg_us": avg_ms * 1e3, "peak_source": peaks.get("_source")}
+            "traffic": measured_traffic("prefill"), "algorithmic_flops": flops,
+            "kernel": f"prefill_kernel (+ activation pre-pass) via matq_linear (gate 14336x4096, r={r}, M={M})",
+            "avg_us": avg_ms * 1e3, "launches_timed": n, "peak_source": peaks.get("_source")}
 
 
 def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
@@ -443,7 +493,7 @@ def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
         torch.cuda.synchronize()
     ms = max_over_ranks(world, e0.elapsed_time(e1), dev) / args.steps
     b, f = step_units(spec)
-    v = (b * world / (ms * 1e-3) / 1e9) if spec["unit"] == "GB/s" else (f * world / (ms * 1e-3) / 1e12)
+    v = whole_job_value(spec["unit"], b, f, world, ms)
     return {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms}
 
