@@ -349,20 +349,24 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
           } else {
             bool arrived = true;
             if (lane == 0) {
+              // acquire load: the contributors' partial sums (published by their fence +
+              // increment) are visible to this warp's loads below, with no further fence
               const int want = (int)(cl - cf);
-              const long long t0 = clock64();
-              while (atomicAdd(cnt, 0) < want) {
-                if (clock64() - t0 > kWaitCycles) {
-                  atomicOr(P.err, 128);
-                  arrived = false;
-                  break;
+              if (ld_acquire_gpu(cnt) < want) {
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(cnt) < want) {
+                  if (clock64() - t0 > kWaitCycles) {
+                    atomicOr(P.err, 128);
+                    arrived = false;
+                    break;
+                  }
+                  __nanosleep(32);
                 }
-                __nanosleep(64);
               }
-              atomicExch(cnt, 0);  // leave the counter at zero for the next call
+              *reinterpret_cast<volatile int*>(cnt) = 0;  // leave the counter at zero for the next call
             }
             arrived = __shfl_sync(0xffffffffu, arrived ? 1 : 0, 0) != 0;
-            __threadfence();
+            __syncwarp();  // orders the other lanes' loads after lane 0's acquire
             float4 acc[RPW * NT];
 #pragma unroll
             for (int j = 0; j < RPW; ++j)
