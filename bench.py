@@ -395,7 +395,7 @@ _KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
 NCU_TRAFFIC = {
-    "decode": {"sha256": None, "bytes": None},
+    "decode": {"sha256": "52308311e012583fe81a02bff60410ed9cf3b5326114be8a9f53d4e6a008bb60", "bytes": 16_120_576 + 0},
     "prefill": {"sha256": "a5e3008895282b04070e43528239556d29fe4623998745f67f56acc196650174", "bytes": 51_869_952 + 31_986_432},
 }
 
