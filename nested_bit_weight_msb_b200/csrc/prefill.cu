@@ -7,15 +7,16 @@
 //   * warp 0 (one thread) streams, with TMA, the raw planes of width r for a 128-row x
 //     256-input block (only those planes: exactly r bits per weight cross HBM) and the fp16
 //     activation tiles [BN tokens x 64 inputs] (128-byte swizzle, the UMMA K-major layout);
-//   * warps 4..7 turn each 64-input slice of the raw planes into an fp16 weight tile
-//     [128 x 64] in shared memory: operand registers are built from the plane words exactly
+//   * warps 4..11 (one 16-row tile each) turn each 64-input slice of the raw planes into an
+//     fp16 weight tile [128 x 64] in shared memory: operand registers are built from the plane words exactly
 //     as on the decode path (1024 + sigma*v), the exact code difference q_hat - z is formed
 //     in fp16 (exact: a half-integer below 256 in magnitude), and one fp16 multiply by the
 //     scale gives W_hat with a single rounding.  stmatrix writes the tiles in the swizzled
 //     layout; fence.proxy.async hands them to the tensor core;
 //   * warp 1 (one thread) issues tcgen05.mma (M = 128 weight rows, N = BN tokens, K = 16)
 //     accumulating in TMEM, and releases ring slots with tcgen05.commit;
-//   * warps 4..7 then read the fp32 accumulator with tcgen05.ld and store y.
+//   * warps 4..11 then read the fp32 accumulator with tcgen05.ld (warp w: TMEM lanes of
+//     quarter w % 4, half of the token columns each) and store y.
 //
 // fp16 (not bf16) weight tiles: with bf16 y, bf16-rounded weights exceed the 2e-3 relative
 // error budget while fp16 ones stay at the output-rounding level; both formats run at the
@@ -39,7 +40,10 @@ constexpr int kSubK = 64;       // inputs per A/B ring slot (one 128-byte swizzl
 constexpr int kRawStages = 2;   // raw-plane ring (256 inputs per slot)
 constexpr int kAStages = 3;     // fp16 weight-tile ring
 constexpr int kBStages = 3;     // activation-tile ring
-constexpr int kThreads = 256;
+constexpr int kDeqWarps = 8;                   // dequantising (and epilogue) warps 4 .. 4 + kDeqWarps - 1
+constexpr int kWarpsPerTile = kDeqWarps >= 8 ? kDeqWarps / 8 : 1;  // warps sharing a 16-row tile
+constexpr int kTilesPerWarp = kDeqWarps >= 8 ? 1 : 8 / kDeqWarps;  // 16-row tiles per warp
+constexpr int kThreads = 32 * (4 + kDeqWarps);
 constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
 
 // ---- activation conversion -----------------------------------------------------------------
@@ -167,29 +171,61 @@ __device__ __forceinline__ void dequant_block(const LaneWords& L, const __half2 
   }
 }
 
-template <int R, int BN, int GROUP, int Q>
-__device__ __forceinline__ void dequant_substage(const LaneWords (&L)[2], const PrefillParams& P, int kc, int rt0,
-                                                 int wq, int lane, uint32_t a_slot) {
+// Scale bits and zero points of one 256-input chunk for a lane's rows (gid, gid + 8 of each of
+// its row tiles), NG = 256 / GROUP groups; loaded before the chunk's planes are waited for.
+template <int GROUP>
+struct ChunkMeta {
+  static constexpr int NG = kChunk / GROUP;
+  uint32_t sb[kTilesPerWarp][NG][2];
+  uint32_t zb[kTilesPerWarp][NG][2];
+};
+
+template <int GROUP>
+__device__ __forceinline__ void load_chunk_meta(ChunkMeta<GROUP>& m, const PrefillParams& P, int kc, int rt0, int wq,
+                                                int lane) {
   const int gid = lane >> 2;
-  const int gi = (kc * kChunk + Q * kSubK) / GROUP;
-  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
 #pragma unroll
-  for (int tt = 0; tt < 2; ++tt) {
-    const int t = 2 * wq + tt;
+  for (int tt = 0; tt < kTilesPerWarp; ++tt)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = (rt0 + kTilesPerWarp * (wq / kWarpsPerTile) + tt) * kTileRows + gid + 8 * h;
+#pragma unroll
+      for (int g = 0; g < ChunkMeta<GROUP>::NG; ++g) {
+        m.sb[tt][g][h] = 0u;
+        m.zb[tt][g][h] = 0u;
+        if (row < P.N) {
+          const size_t o = (size_t)row * P.G + (size_t)kc * ChunkMeta<GROUP>::NG + g;
+          m.sb[tt][g][h] = P.scales[o];
+          m.zb[tt][g][h] = P.zeros[o];
+        }
+      }
+    }
+}
+
+template <int R, int BN, int GROUP, int Q>
+__device__ __forceinline__ void dequant_substage(const LaneWords (&L)[kTilesPerWarp], const ChunkMeta<GROUP>& m,
+                                                 int wq, int lane, uint32_t a_slot) {
+  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
+  constexpr int g = (Q * kSubK) / GROUP;  // group of this 64-input slice inside the chunk
+#pragma unroll
+  for (int tt = 0; tt < kTilesPerWarp; ++tt) {
+    const int t = kTilesPerWarp * (wq / kWarpsPerTile) + tt;
     __half2 s2[2], dz2[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int row = (rt0 + t) * kTileRows + gid + 8 * h;
-      float s = 0.f, zf = 0.f;
-      if (row < P.N) {
-        s = __half2float(__ushort_as_half(P.scales[(size_t)row * P.G + gi]));
-        zf = (float)P.zeros[(size_t)row * P.G + gi];
-      }
-      s2[h] = __float2half2_rn(s);
+      const float sv = __half2float(__ushort_as_half((unsigned short)m.sb[tt][g][h]));
+      const float zf = (float)m.zb[tt][g][h];
+      s2[h] = __float2half2_rn(sv);
       dz2[h] = __float2half2_rn(R == 8 ? zf : (kDelta - zf));
     }
-    dequant_block<R, 2 * Q>(L[tt], s2, dz2, a_slot, t, lane);
-    dequant_block<R, 2 * Q + 1>(L[tt], s2, dz2, a_slot, t, lane);
+    if constexpr (kWarpsPerTile == 1) {
+      dequant_block<R, 2 * Q>(L[tt], s2, dz2, a_slot, t, lane);
+      dequant_block<R, 2 * Q + 1>(L[tt], s2, dz2, a_slot, t, lane);
+    } else if (wq % 2 == 0) {
+      dequant_block<R, 2 * Q>(L[tt], s2, dz2, a_slot, t, lane);
+    } else {
+      dequant_block<R, 2 * Q + 1>(L[tt], s2, dz2, a_slot, t, lane);
+    }
   }
 }
 
@@ -220,8 +256,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   constexpr int kNumPlanes = planes_for_width(R);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRawStages; ++i) { mbar_init(&raw_full[i], 1); mbar_init(&raw_empty[i], 4); }
-    for (int i = 0; i < kAStages; ++i) { mbar_init(&a_full[i], 128); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < kRawStages; ++i) { mbar_init(&raw_full[i], 1); mbar_init(&raw_empty[i], kDeqWarps); }
+    for (int i = 0; i < kAStages; ++i) { mbar_init(&a_full[i], 32 * kDeqWarps); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < kBStages; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
     mbar_init(acc_full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -288,14 +324,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     // ---------------- dequantisation, then epilogue ----------------
     const int wq = warp - 4;
     bool ok = true;
+    ChunkMeta<GROUP> meta;
+    load_chunk_meta<GROUP>(meta, P, 0, rt0, wq, lane);
     for (int kc = 0; kc < KC && ok; ++kc) {
       const int rs = kc % kRawStages;
+      if (kc > 0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
       ok = mbar_wait(&raw_full[rs], (kc / kRawStages) & 1, P.err, 16);
       if (!ok) break;
       const uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
-      LaneWords L[2];
-      lds_lane_words<R>(raw, 2 * wq, lane, L[0]);
-      lds_lane_words<R>(raw, 2 * wq + 1, lane, L[1]);
+      LaneWords L[kTilesPerWarp];
+#pragma unroll
+      for (int tt = 0; tt < kTilesPerWarp; ++tt)
+        lds_lane_words<R>(raw, kTilesPerWarp * (wq / kWarpsPerTile) + tt, lane, L[tt]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&raw_empty[rs]);
 #define MATQ_SUBSTAGE(Q)                                                                       \
@@ -304,7 +344,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
         ok = mbar_wait(&a_empty[as], ((i / kAStages) & 1) ^ 1, P.err, 32);                     \
         if (ok) {                                                                              \
           const uint32_t a_slot = smem_u32(smem + S::kA + as * kATileBytes);                   \
-          dequant_substage<R, BN, GROUP, Q>(L, P, kc, rt0, wq, lane, a_slot);                  \
+          dequant_substage<R, BN, GROUP, Q>(L, meta, wq, lane, a_slot);                        \
           fence_proxy_async();                                                                 \
           mbar_arrive(&a_full[as]);                                                            \
         }                                                                                      \
@@ -312,14 +352,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       MATQ_SUBSTAGE(0) MATQ_SUBSTAGE(1) MATQ_SUBSTAGE(2) MATQ_SUBSTAGE(3)
 #undef MATQ_SUBSTAGE
     }
-    // epilogue: TMEM lanes 32*wq .. 32*wq+31 hold weight rows n0 + 32*wq + lane
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (weight rows n0 + 32*(w%4) + lane);
+    // the warp quads split the BN accumulator columns
     if (ok) ok = mbar_wait(acc_full, 0, P.err, 64);
     if (ok) {
       tc_fence_after();
-      const int n = n0 + 32 * wq + lane;
-      const uint32_t taddr = tmem_d + ((uint32_t)(32 * wq) << 16);
+      const int q = warp & 3, half = wq >> 2;
+      constexpr int kQuads = (kDeqWarps / 4 < BN / 32) ? kDeqWarps / 4 : BN / 32;
+      constexpr int kChunksPerQuad = BN / 32 / kQuads;
+      const int n = n0 + 32 * q + lane;
+      const uint32_t taddr = tmem_d + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * kChunksPerQuad; half < kQuads && c < (half + 1) * kChunksPerQuad; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
         if (n < P.N) {
