@@ -476,13 +476,20 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         tma_load_2d(st + item_plane_off<RG>(p), maps[p], kc * plane_bits(p) * 64, rg * RG, &full[s]);
     }
   };
-  // Activation rows (a bulk copy per token), scales and zero points (cp.async, one row per
-  // streamer thread) of item n; called by the streamer threads (warps 0..7) only.
-  auto stream_rest = [&](int n, int rg, int kc) {
+  // Activation rows of item n: a bulk copy per token (counted in the bytes expected above).
+  auto stream_x = [&](int n, int kc) {
+    const int s = n % kDecStages;
+    const int t = threadIdx.x;
+    if (t < mrows)
+      bulk_load(smem + s * Lt::kStage + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk,
+                kChunk * 2, &full[s]);
+  };
+  // Scales and zero points (cp.async, one row per streamer thread) of item n, and the
+  // streamers' arrivals; called by the streamer threads (warps 0..7) only.
+  auto stream_meta = [&](int n, int rg, int kc) {
     const int s = n % kDecStages;
     uint8_t* st = smem + s * Lt::kStage;
     const int t = threadIdx.x;
-    if (t < mrows) bulk_load(st + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk, kChunk * 2, &full[s]);
     // scales (NG fp16) and the aligned 4-byte word of zeros holding this chunk's NG bytes.
     // The word never crosses the end of the zeros array except when its NG = 2 bytes are the
     // array's last two and start a word; that row is copied with a plain 2-byte load.
@@ -510,21 +517,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   };
   auto refill = [&](int n, int rg, int kc) {
     stream_planes(n, rg, kc);
-    stream_rest(n, rg, kc);
+    stream_x(n, kc);
+    stream_meta(n, rg, kc);
   };
 
+  // Prologue: the weights of the first S items (planes, scales, zero points) depend on no
+  // earlier kernel and are requested at once; the activations after the wait.
   const int pre = nitems < kDecStages ? nitems : kDecStages;
   const int rg0 = (int)(ib / P.KC), kc0 = (int)(ib - (long long)rg0 * P.KC);
   for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
     stream_planes(n, rg, kc);
+    stream_meta(n, rg, kc);
     if (++kc == P.KC) { kc = 0; ++rg; }
   }
   pdl_wait();  // activations, counters and y belong to earlier kernels in the stream
-  if (warp < 8)
-    for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
-      stream_rest(n, rg, kc);
-      if (++kc == P.KC) { kc = 0; ++rg; }
-    }
+  for (int n = 0, kc = kc0; n < pre; ++n) {
+    stream_x(n, kc);
+    if (++kc == P.KC) kc = 0;
+  }
 
   const int rs = warp & 3, ks = warp >> 2;
   if constexpr (Lt::KSL == 2) {
