@@ -3,10 +3,9 @@
 Workload (default, ``--workload ffn8b_decode``): the Llama-3.1-8B-shaped FFN at decode
 batch sizes.  One step runs, for every width r in {2, 3, 4, 6, 8} and every batch
 M in {1, 4, 16}, one FFN forward through the sliced linears:
-    gate = x . W_gate,r^T   [M, 14336]      (matq_linear, decode path)
-    up   = x . W_up,r^T     [M, 14336]
-    a    = silu(gate) * up                  (matq_silu_mul)
-    y    = a . W_down,r^T   [M, 4096]
+    gu   = x . [W_gate; W_up]_r^T   [M, 28672]   (one matq_linear call: gate and up share x)
+    a    = silu(gu[:, :14336]) * gu[:, 14336:]  (matq_silu_mul_gu)
+    y    = a . W_down,r^T           [M, 4096]
 with group-128 parent codes of N(0, 0.02) weights (synthetic, seeded) and N(0, 1) bf16
 activations.  ``value`` = algorithmic bytes of the sliced linears (planes of width r,
 fp16 scales, uint8 zeros, x, y) over the device time of the step -> GB/s.
@@ -73,12 +72,16 @@ def linear_bytes(M, N, K, r, group=GROUP):
     return N * K * r // 8 + N * G * 3 + M * K * 2 + M * N * 2
 
 
+# the sliced-linear calls of one FFN: fused gate+up, then down
+FFN_CALLS = (("gate_up", (2 * D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))
+
+
 def step_units(spec):
     """(algorithmic bytes, flops) of one step."""
     b = f = 0
     for r in spec["widths"]:
         for M in spec["batches"]:
-            for (N, K) in ((D_FF, D_MODEL), (D_FF, D_MODEL), (D_MODEL, D_FF)):
+            for _, (N, K) in FFN_CALLS:
                 b += linear_bytes(M, N, K, r)
                 f += 2 * M * N * K
     return b, f
@@ -227,6 +230,13 @@ def host_weights():
             for name, (N, K) in (("gate", (D_FF, D_MODEL)), ("up", (D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))}
 
 
+def fused_weights(w):
+    """gate and up read the same x: their codes, scales and zero points are stacked along N
+    into one [2F, D] matrix served by one call."""
+    gu = tuple(np.concatenate([w["gate"][i], w["up"][i]], axis=0) for i in range(3))
+    return {"gate_up": gu, "down": w["down"]}
+
+
 # ---------------------------------------------------------------------------------------------
 # reference arm: the oracle on the host
 # ---------------------------------------------------------------------------------------------
@@ -278,7 +288,7 @@ def run_ours(args):
     # pack once per matrix (one-time), then clone into rotating copies
     packed = {}
     meta = {}
-    for name, (q, s, z) in weights.items():
+    for name, (q, s, z) in fused_weights(weights).items():
         dq = torch.from_numpy(q).to(dev)
         p = matq.pack(dq, r_keep=8)
         packed[name] = [p] + [p.clone() for _ in range(args.copies - 1)]
@@ -292,10 +302,9 @@ def run_ours(args):
         xb, _ = synth.activations(M, D_MODEL, seed=rank, outlier_frac=spec["outlier"])
         xs[M] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
     Mmax = max(batches)
-    ws = torch.zeros(max(matq.workspace_bytes(Mmax, D_FF, D_FF, GROUP), matq.workspace_bytes(Mmax, D_MODEL, D_FF, GROUP)),
+    ws = torch.zeros(max(matq.workspace_bytes(Mmax, K, N, GROUP) for _, (N, K) in FFN_CALLS),
                      dtype=torch.uint8, device=dev)
-    gate_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
-    up_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
+    gu_buf = {M: torch.empty((M, 2 * D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
     a_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
     y_buf = {M: torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev) for M in batches}
 
@@ -304,9 +313,8 @@ def run_ours(args):
         matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, workspace=ws)
 
     def ffn(x, M, r, copy):
-        linear("gate", copy, x, r, gate_buf[M])
-        linear("up", copy, x, r, up_buf[M])
-        matq.silu_mul(gate_buf[M], up_buf[M], out=a_buf[M])
+        linear("gate_up", copy, x, r, gu_buf[M])
+        matq.silu_mul_gu(gu_buf[M], out=a_buf[M])
         linear("down", copy, a_buf[M], r, y_buf[M])
 
     calls = [(r, M) for r in spec["widths"] for M in batches]
@@ -343,7 +351,7 @@ def run_ours(args):
     value = whole_job_value(spec["unit"], b, f, world, ms_step)
 
     # ---- roofline of the dominant kernel: per-call device time of the sliced linear ----------
-    rl = roofline(args, spec, linear, xs, gate_buf, stream, dev)
+    rl = roofline(args, spec, linear, xs, gu_buf, stream, dev)
 
     # ---- end-to-end through the public API with host buffers --------------------------------
     e2e = end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world)
@@ -355,15 +363,16 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16-operands/f32-acc (bf16 in/out)", "data": "synthetic",
-            "config": {"workload": args.workload, "shapes": "gate/up [14336,4096], down [4096,14336], group 128",
+            "config": {"workload": args.workload,
+                       "shapes": "gate+up fused [28672,4096] (two [14336,4096] stacked), down [4096,14336], group 128",
                        "widths": list(spec["widths"]), "batches": list(batches),
                        "l2": f"rotating {args.copies} device copies of the packed layer (> L2)",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graph replay, CUDA events"},
             "roofline": rl,
             "e2e": e2e,
-            # per FFN: gate, up, down (one kernel each on the decode path, conversion + GEMM on
-            # the prefill path) and the SiLU-gated product
-            "gpu_launches": args.steps * len(calls) * (3 * (1 if spec["unit"] == "GB/s" else 2) + 1),
+            # per FFN: fused gate+up and down (one kernel each on the decode path, conversion +
+            # GEMM on the prefill path) and the SiLU-gated product
+            "gpu_launches": args.steps * len(calls) * (len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2) + 1),
             "clocks": clk.summary(),
             "peaks_source": peaks.get("_source"),
         }
@@ -394,9 +403,11 @@ _KERNEL_SOURCES = {
     "decode": ("decode.cu", "common.cuh", "operands.cuh", "sync.cuh"),
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
-NCU_TRAFFIC = {
-    "decode": {"sha256": "52308311e012583fe81a02bff60410ed9cf3b5326114be8a9f53d4e6a008bb60", "bytes": 16_120_576 + 0},
-    "prefill": {"sha256": "a5e3008895282b04070e43528239556d29fe4623998745f67f56acc196650174", "bytes": 51_869_952 + 31_986_432},
+NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
+    "decode": {"sha256": "ce5c2fda4d7f9c5ecb8cc359341805ebc97ebf5297651e0a555a94ad62b1cca0", "launch": "gate_up 28672x4096 r=2 M=1",
+               "bytes": 32_177_920 + 0},
+    "prefill": {"sha256": "7ef9fa1fc301969c4e1efa3dd5d4abd701a39fe5872f0a06657a8dcdb5d07be4", "launch": "gate_up 28672x4096 r=4 M=2048",
+                "bytes": 186_167_552 + 96_039_936},
 }
 
 
@@ -409,14 +420,14 @@ def kernel_source_sha(path_kind):
     return h.hexdigest()
 
 
-def measured_traffic(path_kind):
+def measured_traffic(path_kind, launch):
     rec = NCU_TRAFFIC[path_kind]
-    if rec["bytes"] is None or rec["sha256"] != kernel_source_sha(path_kind):
+    if rec["bytes"] is None or rec.get("launch") != launch or rec["sha256"] != kernel_source_sha(path_kind):
         return None
     return rec["bytes"]
 
 
-def roofline(args, spec, linear, xs, gate_buf, stream, dev):
+def roofline(args, spec, linear, xs, gu_buf, stream, dev):
     """Average device time per launch of the dominant kernel in steady state: a CUDA graph of
     back-to-back sliced-linear calls on the gate matrix (rotating weight copies, so every call
     streams from HBM), timed with CUDA events on the launching stream; total / launches."""
@@ -427,12 +438,12 @@ def roofline(args, spec, linear, xs, gate_buf, stream, dev):
     n = 24
     with torch.cuda.stream(stream):
         for i in range(3):
-            linear("gate", i % args.copies, xs[M], r, gate_buf[M])
+            linear("gate_up", i % args.copies, xs[M], r, gu_buf[M])
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
-                linear("gate", i % args.copies, xs[M], r, gate_buf[M])
+                linear("gate_up", i % args.copies, xs[M], r, gu_buf[M])
         g.replay()
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -446,20 +457,22 @@ def roofline(args, spec, linear, xs, gate_buf, stream, dev):
             reps.append(e0.elapsed_time(e1) / n)
     del g
     avg_ms = float(np.median(reps))
+    N = 2 * D_FF
+    launch = f"gate_up {N}x{D_MODEL} r={r} M={M}"
     if spec["unit"] == "GB/s":
-        units = linear_bytes(M, D_FF, D_MODEL, r)
+        units = linear_bytes(M, N, D_MODEL, r)
         ach = units / (avg_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": measured_traffic("decode"), "algorithmic_bytes": units,
-                "kernel": f"decode_kernel via matq_linear (gate 14336x4096, r={r}, M={M})",
+                "traffic": measured_traffic("decode", launch), "algorithmic_bytes": units,
+                "kernel": f"decode_kernel via matq_linear ({launch})",
                 "avg_us": avg_ms * 1e3, "launches_timed": n, "peak_source": peaks.get("_source")}
-    flops = 2 * M * D_FF * D_MODEL
+    flops = 2 * M * N * D_MODEL
     ach = flops / (avg_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-            "traffic": measured_traffic("prefill"), "algorithmic_flops": flops,
-            "kernel": f"prefill_kernel (+ activation pre-pass) via matq_linear (gate 14336x4096, r={r}, M={M})",
+            "traffic": measured_traffic("prefill", launch), "algorithmic_flops": flops,
+            "kernel": f"prefill_kernel (+ activation pre-pass) via matq_linear ({launch})",
             "avg_us": avg_ms * 1e3, "launches_timed": n, "peak_source": peaks.get("_source")}
 
 
@@ -499,22 +512,23 @@ def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
 
 
 def run_case(args):
-    """A few single calls of the gate projection (14336 x 4096, group 128) at width r and
-    batch m, rotating through device copies of the pack (> L2); used for ncu captures."""
+    """A few single calls of the fused gate+up projection (28672 x 4096, group 128) at width r
+    and batch m, rotating through device copies of the pack (> L2); used for ncu captures."""
     import torch
     from nested_bit_weight_msb_b200 import matq, synth
     torch.cuda.set_device(0)
-    q, s, z = synth.parent_weights(D_FF, D_MODEL, GROUP, seed=0, proj="gate")
+    q, s, z = fused_weights(host_weights())["gate_up"]
+    N = q.shape[0]
     p0 = matq.pack(torch.from_numpy(q).cuda(), r_keep=8)
     packs = [p0] + [p0.clone() for _ in range(args.copies - 1)]
     ds = torch.from_numpy(s.view(np.int16)).cuda()
     dz = torch.from_numpy(z).cuda()
     xb, _ = synth.activations(args.m, D_MODEL, seed=0, outlier_frac=0.01 if args.case == "prefill" else 0.0)
     dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
-    ws = matq.workspace(args.m, D_MODEL, D_FF, GROUP)
-    y = torch.empty((args.m, D_FF), dtype=torch.bfloat16, device="cuda")
+    ws = matq.workspace(args.m, D_MODEL, N, GROUP)
+    y = torch.empty((args.m, N), dtype=torch.bfloat16, device="cuda")
     for i in range(args.calls):
-        matq.linear(dx, packs[i % len(packs)], 8, ds, dz, D_FF, args.r, GROUP, y=y, workspace=ws)
+        matq.linear(dx, packs[i % len(packs)], 8, ds, dz, N, args.r, GROUP, y=y, workspace=ws)
     torch.cuda.synchronize()
     assert matq.workspace_status(ws) == 0
     print(json.dumps({"case": args.case, "r": args.r, "m": args.m, "calls": args.calls, "ok": True}))

@@ -228,6 +228,13 @@ int matq_rmsnorm(const float* h, int M, int D, float eps, void* n_out, void* str
  *   gate, up, a_out [M, F] bf16. */
 int matq_silu_mul(const void* gate, const void* up, int M, int F, void* a_out, void* stream);
 
+/* The same product for the output of ONE fused gate+up projection (gate and up read the same
+ * x, so their weights can be packed as one [2F, D] matrix and served by one matq_linear call;
+ * "MatGPTQ" §4 applies the sliced kernel per linear layer, this fusion is this library's).
+ *   gu    [M, 2F] bf16: row m holds gate in columns 0..F-1 and up in columns F..2F-1.
+ *   a_out [M, F] bf16: a = bf16( silu(gate) * up ).  F % 8 == 0 takes the vector path. */
+int matq_silu_mul_gu(const void* gu, int M, int F, void* a_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -189,6 +189,15 @@ int matq_rmsnorm(const float* h, int M, int D, float eps, void* n_out, void* str
   return cuda_status(launch_rmsnorm(h, M, D, eps, n_out, (cudaStream_t)stream));
 }
 
+int matq_silu_mul_gu(const void* gu, int M, int F, void* a_out, void* stream) {
+  if (M < 1 || F < 1 || (long long)M * F > (1LL << 40)) return MATQ_EINVAL_SHAPE;
+  if (!gu || !a_out) return MATQ_ENULL;
+  if (!aligned16(gu) || !aligned16(a_out)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_silu_mul_gu(gu, M, F, a_out, (cudaStream_t)stream));
+}
+
 int matq_silu_mul(const void* gate, const void* up, int M, int F, void* a_out, void* stream) {
   if (M < 1 || F < 1 || (long long)M * F > (1LL << 40)) return MATQ_EINVAL_SHAPE;
   if (!gate || !up || !a_out) return MATQ_ENULL;

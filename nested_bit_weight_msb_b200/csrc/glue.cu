@@ -56,6 +56,37 @@ __global__ void __launch_bounds__(256) silu_mul_kernel(const __nv_bfloat16* __re
     out[i] = __float2bfloat16_rn(silu_f(__bfloat162float(gate[i])) * __bfloat162float(up[i]));
 }
 
+// Same product for the output of one fused gate+up projection: gu [M, 2F], row m holding
+// gate in columns 0..F-1 and up in F..2F-1; out [M, F].  Vector path needs F % 8 == 0.
+__global__ void __launch_bounds__(256) silu_mul_gu_kernel(const __nv_bfloat16* __restrict__ gu, int M, int F,
+                                                          __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int stride = gridDim.x * blockDim.x;
+  for (int m = blockIdx.y; m < M; m += gridDim.y) {
+    const __nv_bfloat16* g = gu + (size_t)m * 2 * F;
+    const __nv_bfloat16* u = g + F;
+    __nv_bfloat16* o = out + (size_t)m * F;
+    if ((F & 7) == 0) {
+      for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < F / 8; v += stride) {
+        const uint4 g4 = reinterpret_cast<const uint4*>(g)[v];
+        const uint4 u4 = reinterpret_cast<const uint4*>(u)[v];
+        const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&g4);
+        const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&u4);
+        uint4 o4;
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(&o4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          ob[i] = __float2bfloat16_rn(silu_f(__bfloat162float(gb[i])) * __bfloat162float(ub[i]));
+        reinterpret_cast<uint4*>(o)[v] = o4;
+      }
+    } else {
+      for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < F; i += stride)
+        o[i] = __float2bfloat16_rn(silu_f(__bfloat162float(g[i])) * __bfloat162float(u[i]));
+    }
+  }
+}
+
 cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s) {
   return launch_pdl(rmsnorm_kernel, dim3(M), dim3(256), 0, s, h, D, eps, (__nv_bfloat16*)out);
 }
@@ -70,4 +101,18 @@ cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void
                     (const __nv_bfloat16*)up, n, (__nv_bfloat16*)out);
 }
 
+}  // namespace matq
+
+namespace matq {
+cudaError_t launch_silu_mul_gu(const void* gu, int M, int F, void* out, cudaStream_t s) {
+  const int per_row = ((F & 7) == 0 ? F / 8 : F);
+  int bx = (per_row + 255) / 256;
+  if (bx > 148 * 4) bx = 148 * 4;
+  if (bx < 1) bx = 1;
+  int by = M < 65535 ? M : 65535;
+  // keep the grid near a few waves of the SMs
+  while (by > 1 && (long long)bx * by > 148 * 16) by = (by + 1) / 2;
+  return launch_pdl(silu_mul_gu_kernel, dim3(bx, by), dim3(256), 0, s, (const __nv_bfloat16*)gu, M, F,
+                    (__nv_bfloat16*)out);
+}
 }  // namespace matq

@@ -25,6 +25,7 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
 
 cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s);
 cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s);
+cudaError_t launch_silu_mul_gu(const void* gu, int M, int F, void* out, cudaStream_t s);
 
 // C-ABI status helpers (api.cu): record a failed CUDA call as the thread's last CUDA error and
 // return MATQ_ECUDA; check that the current device is an sm_100 part.

@@ -63,6 +63,7 @@ _SIGNATURES = {
                                      _c_vp, _c_int, _c_vp, _c_vp]),
     "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
     "matq_silu_mul": (_c_int, [_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_vp]),
+    "matq_silu_mul_gu": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_vp]),
 }
 
 for _name, (_res, _args) in _SIGNATURES.items():
@@ -201,4 +202,15 @@ def silu_mul(gate, up, out=None, stream=None):
     if out is None:
         out = torch.empty((M, F), dtype=torch.bfloat16, device=gate.device)
     check(matq_silu_mul(_ptr(gate), _ptr(up), M, F, _ptr(out), _stream_ptr(stream)), "matq_silu_mul")
+    return out
+
+
+def silu_mul_gu(gu, out=None, stream=None):
+    """a = silu(gate) * up from one fused gate+up output gu [M, 2F] (gate = first F columns)."""
+    torch = _torch()
+    M, F2 = gu.shape
+    F = F2 // 2
+    if out is None:
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=gu.device)
+    check(matq_silu_mul_gu(_ptr(gu), M, F, _ptr(out), _stream_ptr(stream)), "matq_silu_mul_gu")
     return out

@@ -117,3 +117,7 @@ def test_glue_rejects(M):
     assert M.matq_rmsnorm(FAKE, 0, 16, 1e-5, FAKE, None) == M.MATQ_EINVAL_SHAPE
     assert M.matq_rmsnorm(None, 1, 16, 1e-5, FAKE, None) == M.MATQ_ENULL
     assert M.matq_silu_mul(FAKE, FAKE + 2, 1, 16, FAKE, None) == M.MATQ_EALIGN
+    assert M.matq_silu_mul_gu(FAKE, 0, 16, FAKE, None) == M.MATQ_EINVAL_SHAPE
+    assert M.matq_silu_mul_gu(FAKE, 1, 0, FAKE, None) == M.MATQ_EINVAL_SHAPE
+    assert M.matq_silu_mul_gu(None, 1, 16, FAKE, None) == M.MATQ_ENULL
+    assert M.matq_silu_mul_gu(FAKE + 2, 1, 16, FAKE, None) == M.MATQ_EALIGN

@@ -51,6 +51,39 @@ def test_silu_mul(M, Mt, F):
     check_close(_bf16(a), O.gated_product(gv, uv), what="silu_mul")
 
 
+@pytest.mark.parametrize("Mt,F", [(1, 14336), (16, 14336), (3, 1001), (5, 24)])
+def test_silu_mul_gu(M, Mt, F):
+    """Gated product read from the two halves of one fused gate+up output [M, 2F]."""
+    import torch
+    rng = np.random.default_rng(F + 7 * Mt)
+    gub, guv = synth.bf16_round((rng.standard_normal((Mt, 2 * F)) * 3).astype(np.float32))
+    gu = torch.from_numpy(gub.view(np.int16)).cuda().view(torch.bfloat16)
+    a = M.silu_mul_gu(gu)
+    check_close(_bf16(a), O.gated_product(guv[:, :F], guv[:, F:]), what="silu_mul_gu")
+
+
+@pytest.mark.parametrize("Mt,r", [(1, 2), (16, 4), (40, 3)])
+def test_fused_gate_up_block(M, Mt, r):
+    """One sliced linear over the row-concatenated [W_gate; W_up] pack, then the gated product
+    from its halves: teacher-forced against the oracle's separate gate and up projections."""
+    import torch
+    D, F, G = 512, 1024, 128
+    host = {name: synth.parent_weights(F, D, G, seed=4, layer=0, proj=name) for name in ("gate", "up")}
+    q = np.concatenate([host["gate"][0], host["up"][0]], axis=0)
+    s = np.concatenate([host["gate"][1], host["up"][1]], axis=0)
+    z = np.concatenate([host["gate"][2], host["up"][2]], axis=0)
+    planes = M.pack(torch.from_numpy(q).cuda(), r_keep=8)
+    xb, xv = synth.activations(Mt, D, seed=6)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    gu = M.linear(x, planes, 8, torch.from_numpy(s.view(np.int16)).cuda(), torch.from_numpy(z).cuda(), 2 * F, r, G)
+    g_ref = O.linear(xv.astype(np.float64), *host["gate"], r, G)
+    u_ref = O.linear(xv.astype(np.float64), *host["up"], r, G)
+    check_close(_bf16(gu)[:, :F], g_ref, what="fused gate half")
+    check_close(_bf16(gu)[:, F:], u_ref, what="fused up half")
+    a = M.silu_mul_gu(gu)
+    check_close(_bf16(a), O.gated_product(_bf16(gu)[:, :F], _bf16(gu)[:, F:]), what="fused gated product")
+
+
 @pytest.mark.parametrize("Mt", [1, 16, 40])
 def test_mixnmatch_stack_teacher_forced(M, Mt):
     import torch
