@@ -52,8 +52,13 @@ constexpr int kRowSlices = 4;        // warps split an item's row tiles four way
 // register budget of a thread stays at 255, and only two code variants share the I-cache)
 __host__ __device__ constexpr int k_slices(int NT) { return NT > 0 ? 2 : 2; }
 __host__ __device__ constexpr int dec_threads(int NT) { return 32 * kRowSlices * k_slices(NT); }
-constexpr int kDecStages = 4;        // ring depth
-constexpr int kMaxDecodeCTAs = 160;  // bound used to size the partial-sum workspace
+// Resident CTAs per SM (CPS): two for M <= 8, r >= 6 on matrices with K <= 4096 (each CTA's 8
+// warps then fit 128 registers a thread, so an SM runs 16 warps and hides more latency; r = 6
+// and 8 carry the most operand-building work per item), otherwise one.  On long-K matrices a
+// row group would be split between too many CTAs; at r <= 4 the gain of the call is lost
+// because two resident CTAs keep the next kernel from starting its prologue early.
+constexpr int kMaxSMs = 160;  // bound on the SMs used, which sizes the partial-sum workspace
+__host__ __device__ constexpr int max_ctas_per_sm(int NT) { return NT == 1 ? 2 : 1; }
 constexpr int kXPitch = kChunk * 2 + 16;  // bytes per activation row in a stage (padded)
 
 __host__ __device__ constexpr int rows_per_warp_tiles(int r) { return r <= 4 ? 4 : 2; }
@@ -70,7 +75,7 @@ struct DecodeParams {
   int* err;
 };
 
-template <int R, int NT, int GROUP>
+template <int R, int NT, int GROUP, int CPS>
 struct DecodeLayout {
   static constexpr int RPW = rows_per_warp_tiles(R);
   static constexpr int RG = kRowSlices * RPW;           // row tiles per item
@@ -86,10 +91,15 @@ struct DecodeLayout {
   static constexpr int kStage = ((oZ + kMetaZ) + 127) & ~127;
   static constexpr int KSL = k_slices(NT);
   static constexpr int kThreads = dec_threads(NT);
-  static constexpr int oRed = kDecStages * kStage;     // k-slice reduction buffer
   static constexpr int kRed = (KSL - 1) * kRowSlices * RPW * NT * 4 * 32 * 4;
+  // ring depth: up to 4 stages within the CTA's share of the SM's shared memory
+  static constexpr int kSmemBudget = CPS == 2 ? 113 * 1024 : 224 * 1024;
+  static constexpr int kStagesFit = (kSmemBudget - kRed - 256) / kStage;
+  static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit < 2 ? 2 : kStagesFit;
+  static constexpr int oRed = kStages * kStage;     // k-slice reduction buffer
   static constexpr int oBar = oRed + kRed;
-  static constexpr int kSmem = oBar + 2 * kDecStages * 8 + 128;
+  static constexpr int kSmem = oBar + 2 * kStages * 8 + 128;
+  static_assert(kSmem <= kSmemBudget, "decode stage ring exceeds the CTA's shared memory");
 };
 
 // plane p's offset inside an item's plane region (RG row tiles each)
@@ -150,11 +160,11 @@ __device__ __forceinline__ long long item_owner(long long u, long long I, long l
 }
 
 // Work of one warp: RPW row tiles (row slice rs) x input slice KS of every item.
-template <int R, int NT, int GROUP, int KS, typename Refill>
+template <int R, int NT, int GROUP, int CPS, int KS, typename Refill>
 __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem, uint64_t* full, uint64_t* empty,
                                             float* red, long long c, long long ib, long long ie, int rs, int lane,
                                             Refill&& refill) {
-  using Lt = DecodeLayout<R, NT, GROUP>;
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
   constexpr int RPW = Lt::RPW, RG = Lt::RG, NG = Lt::NG, KSL = Lt::KSL;
   constexpr int NB = 8 / KSL;                                    // 32-input blocks per slice
   constexpr int kPromoteEvery = (GROUP / 32 < NB) ? GROUP / 32 : NB;  // blocks per scale group part
@@ -190,8 +200,8 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   const int rg_first = (int)(ib / P.KC);
   int rg = rg_first, kc = (int)(ib - (long long)rg_first * P.KC);
   for (int n = 0; n < nitems; ++n) {
-    const int s = n % kDecStages;
-    if (ok) ok = mbar_wait(&full[s], (n / kDecStages) & 1, P.err, 2);
+    const int s = n % Lt::kStages;
+    if (ok) ok = mbar_wait(&full[s], (n / Lt::kStages) & 1, P.err, 2);
     if (ok) {
       const uint8_t* st = smem + s * Lt::kStage;
       LaneWords L[RPW];
@@ -269,15 +279,15 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     // the streaming warps (0..7) refill this slot with item n + S once every warp released it
-    if (rs + kRowSlices * KS < 8 && n + kDecStages < nitems && ok) {
-      ok = mbar_wait(&empty[s], (n / kDecStages) & 1, P.err, 1);
+    if (rs + kRowSlices * KS < 8 && n + Lt::kStages < nitems && ok) {
+      ok = mbar_wait(&empty[s], (n / Lt::kStages) & 1, P.err, 1);
       if (ok) {
-        int rg2 = rg, kc2 = kc + kDecStages;
+        int rg2 = rg, kc2 = kc + Lt::kStages;
         while (kc2 >= P.KC) {
           kc2 -= P.KC;
           ++rg2;
         }
-        refill(n + kDecStages, rg2, kc2);
+        refill(n + Lt::kStages, rg2, kc2);
       }
     }
 
@@ -374,7 +384,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
               for (int nt = 0; nt < NT; ++nt)
                 acc[j * NT + nt] = make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
             // the other contributors in CTA order (deterministic); kU at a time so loads overlap
-            constexpr int kU = (RPW * NT >= 8) ? 2 : (16 / (RPW * NT));
+            constexpr int kU = CPS == 2 ? 1 : (RPW * NT >= 8) ? 2 : (16 / (RPW * NT));
             for (long long c2 = cf + 1; arrived && c2 <= cl; c2 += kU) {
               float4 v[kU][RPW * NT];
 #pragma unroll
@@ -427,12 +437,12 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   }
 }
 
-template <int R, int NT, int GROUP>
-__global__ void __launch_bounds__(dec_threads(NT), 1)
+template <int R, int NT, int GROUP, int CPS>
+__global__ void __launch_bounds__(dec_threads(NT), CPS)
 decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
               const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tm3,
               const __grid_constant__ CUtensorMap tm4, const DecodeParams P) {
-  using Lt = DecodeLayout<R, NT, GROUP>;
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
   constexpr int RG = Lt::RG, NG = Lt::NG, NTOK = Lt::NTOK;
   constexpr int kNumPlanes = planes_for_width(R);
   constexpr int kThreads = Lt::kThreads;
@@ -440,7 +450,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
 
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lt::oBar);
-  uint64_t* empty = full + kDecStages;
+  uint64_t* empty = full + Lt::kStages;
   float* red = reinterpret_cast<float*>(smem + Lt::oRed);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -451,14 +461,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   const int mrows = P.M < NTOK ? P.M : NTOK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < Lt::kStages; ++s) {
       mbar_init(&full[s], 1 + kStreamers);  // thread 0's arrival + one arrival per streamer
       mbar_init(&empty[s], kThreads / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // activation rows >= M stay zero in every stage (nothing is ever copied there)
-  for (int s = 0; s < kDecStages; ++s)
+  for (int s = 0; s < Lt::kStages; ++s)
     for (int i = threadIdx.x; i < (NTOK - mrows) * kXPitch / 4; i += kThreads)
       reinterpret_cast<uint32_t*>(smem + s * Lt::kStage + Lt::oX + mrows * kXPitch)[i] = 0u;
   __syncthreads();
@@ -468,7 +478,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   // Planes of item n into slot n % S (2-D TMA by thread 0): they depend on no earlier kernel.
   auto stream_planes = [&](int n, int rg, int kc) {
     if (threadIdx.x == 0) {
-      const int s = n % kDecStages;
+      const int s = n % Lt::kStages;
       uint8_t* st = smem + s * Lt::kStage;
       mbar_expect_tx_only(&full[s], Lt::kPlanes + mrows * kChunk * 2);
 #pragma unroll
@@ -478,7 +488,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   };
   // Activation rows of item n: a bulk copy per token (counted in the bytes expected above).
   auto stream_x = [&](int n, int kc) {
-    const int s = n % kDecStages;
+    const int s = n % Lt::kStages;
     const int t = threadIdx.x;
     if (t < mrows)
       bulk_load(smem + s * Lt::kStage + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk,
@@ -487,7 +497,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   // Scales and zero points (cp.async, one row per streamer thread) of item n, and the
   // streamers' arrivals; called by the streamer threads (warps 0..7) only.
   auto stream_meta = [&](int n, int rg, int kc) {
-    const int s = n % kDecStages;
+    const int s = n % Lt::kStages;
     uint8_t* st = smem + s * Lt::kStage;
     const int t = threadIdx.x;
     // scales (NG fp16) and the aligned 4-byte word of zeros holding this chunk's NG bytes.
@@ -523,7 +533,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
 
   // Prologue: the weights of the first S items (planes, scales, zero points) depend on no
   // earlier kernel and are requested at once; the activations after the wait.
-  const int pre = nitems < kDecStages ? nitems : kDecStages;
+  const int pre = nitems < Lt::kStages ? nitems : Lt::kStages;
   const int rg0 = (int)(ib / P.KC), kc0 = (int)(ib - (long long)rg0 * P.KC);
   for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
     stream_planes(n, rg, kc);
@@ -537,17 +547,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   }
 
   const int rs = warp & 3, ks = warp >> 2;
-  if constexpr (Lt::KSL == 2) {
-    if (ks == 0) decode_warp<R, NT, GROUP, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
-    else decode_warp<R, NT, GROUP, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
-    return;
-  }
-  switch (ks) {
-    case 0: decode_warp<R, NT, GROUP, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
-    case 1: decode_warp<R, NT, GROUP, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
-    case 2: decode_warp<R, NT, GROUP, 2>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
-    default: decode_warp<R, NT, GROUP, 3>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill); break;
-  }
+  static_assert(Lt::KSL == 2, "two input slices per item");
+  if (ks == 0) decode_warp<R, NT, GROUP, CPS, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+  else decode_warp<R, NT, GROUP, CPS, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
 }
 
 // ---- host side -----------------------------------------------------------------------------
@@ -561,7 +563,8 @@ long long max_decode_rows() { return (long long)(kHeaderCounters / kRowSlices) *
 
 size_t decode_workspace_bytes(int M) {
   const int NT = (M <= 8) ? 1 : 2;
-  const size_t partial = (size_t)2 * kMaxDecodeCTAs * kRowSlices * 4 * NT * 4 * 32 * sizeof(float);
+  const size_t partial =
+      (size_t)2 * kMaxSMs * max_ctas_per_sm(NT) * kRowSlices * 4 * NT * 4 * 32 * sizeof(float);
   return kHeaderBytes + ((partial + 255) & ~size_t(255));
 }
 
@@ -591,10 +594,10 @@ static cudaError_t plane_map(CUtensorMap* m, const uint8_t* base, const PlaneGeo
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int R, int NT, int GROUP>
+template <int R, int NT, int GROUP, int CPS>
 static cudaError_t launch_decode_t(const uint8_t* planes, const PlaneGeom& g, DecodeParams P, int sms,
                                    cudaStream_t s) {
-  using Lt = DecodeLayout<R, NT, GROUP>;
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
   CUtensorMap maps[5];
   for (int p = 0; p < 5; ++p) {
     if (p < planes_for_width(R)) {
@@ -606,23 +609,24 @@ static cudaError_t launch_decode_t(const uint8_t* planes, const PlaneGeom& g, De
   }
   P.NRG = (g.RT + Lt::RG - 1) / Lt::RG;
   P.I = (long long)P.NRG * g.KC;
-  P.C = (int)(P.I < sms ? P.I : sms);
-  auto kern = decode_kernel<R, NT, GROUP>;
+  const long long ctas = (long long)sms * CPS;
+  P.C = (int)(P.I < ctas ? P.I : ctas);
+  auto kern = decode_kernel<R, NT, GROUP, CPS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(P.C), dim3(Lt::kThreads), (size_t)Lt::kSmem, s, maps[0], maps[1], maps[2], maps[3],
                     maps[4], P);
 }
 
-template <int NT, int GROUP>
+template <int NT, int GROUP, int CPS>
 static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom& g, const DecodeParams& P, int sms,
                                    cudaStream_t s) {
   switch (r) {
-    case 2: return launch_decode_t<2, NT, GROUP>(planes, g, P, sms, s);
-    case 3: return launch_decode_t<3, NT, GROUP>(planes, g, P, sms, s);
-    case 4: return launch_decode_t<4, NT, GROUP>(planes, g, P, sms, s);
-    case 6: return launch_decode_t<6, NT, GROUP>(planes, g, P, sms, s);
-    default: return launch_decode_t<8, NT, GROUP>(planes, g, P, sms, s);
+    case 2: return launch_decode_t<2, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 3: return launch_decode_t<3, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 4: return launch_decode_t<4, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 6: return launch_decode_t<6, NT, GROUP, CPS>(planes, g, P, sms, s);
+    default: return launch_decode_t<8, NT, GROUP, CPS>(planes, g, P, sms, s);
   }
 }
 
@@ -634,7 +638,7 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (sms > kMaxDecodeCTAs) sms = kMaxDecodeCTAs;
+  if (sms > kMaxSMs) sms = kMaxSMs;
   DecodeParams P;
   P.N = g.N;
   P.K = K;
@@ -651,9 +655,11 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
   P.partial = (float*)(ws + kHeaderBytes);
   P.y = y;
   const uint8_t* pl = (const uint8_t*)planes;
+  if (NT == 1 && g.KC <= 16)
+    return group == 64 ? launch_decode_r<1, 64, 2>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 2>(r, pl, g, P, sms, s);
   if (NT == 1)
-    return group == 64 ? launch_decode_r<1, 64>(r, pl, g, P, sms, s) : launch_decode_r<1, 128>(r, pl, g, P, sms, s);
-  return group == 64 ? launch_decode_r<2, 64>(r, pl, g, P, sms, s) : launch_decode_r<2, 128>(r, pl, g, P, sms, s);
+    return group == 64 ? launch_decode_r<1, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 1>(r, pl, g, P, sms, s);
+  return group == 64 ? launch_decode_r<2, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<2, 128, 1>(r, pl, g, P, sms, s);
 }
 
 }  // namespace matq
