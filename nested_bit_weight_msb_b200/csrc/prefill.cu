@@ -249,9 +249,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rt0 = blockIdx.x * (kBM / kTileRows);
-  const int n0 = blockIdx.x * kBM;
-  const int m0 = blockIdx.y * BN;
+  // token tiles are the fastest grid dimension: the CTAs of one weight-row block run together
+  // and share its planes through L2
+  const int rt0 = blockIdx.y * (kBM / kTileRows);
+  const int n0 = blockIdx.y * kBM;
+  const int m0 = blockIdx.x * BN;
   const int KC = P.K / kChunk;
   constexpr int kNumPlanes = planes_for_width(R);
 
@@ -422,7 +424,7 @@ static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P
   auto kern = prefill_kernel<R, BN, GROUP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
   if (e != cudaSuccess) return e;
-  dim3 grid((P.N + kBM - 1) / kBM, (P.M + BN - 1) / BN);
+  dim3 grid((P.M + BN - 1) / BN, (P.N + kBM - 1) / kBM);
   return launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3], maps[4],
                     maps[5], P);
 }
