@@ -4,19 +4,22 @@
 // Efficient and Accurate Inference over Nested Quantized Models", App. A.1 and §4).  This
 // path is a dense contraction, so it runs on the 5th-generation tensor cores:
 //
+//   * one persistent CTA per SM takes output tiles [128 weight rows x BN tokens] in turn
+//     (token tiles fastest, so the CTAs on one weight-row block share its planes in L2);
 //   * warp 0 (one thread) streams, with TMA, the raw planes of width r for a 128-row x
 //     256-input block (only those planes: exactly r bits per weight cross HBM) and the fp16
 //     activation tiles [BN tokens x 64 inputs] (128-byte swizzle, the UMMA K-major layout);
 //   * warps 4..11 (one 16-row tile each) turn each 64-input slice of the raw planes into an
-//     fp16 weight tile [128 x 64] in shared memory: operand registers are built from the plane words exactly
-//     as on the decode path (1024 + sigma*v), the exact code difference q_hat - z is formed
-//     in fp16 (exact: a half-integer below 256 in magnitude), and one fp16 multiply by the
-//     scale gives W_hat with a single rounding.  stmatrix writes the tiles in the swizzled
-//     layout; fence.proxy.async hands them to the tensor core;
+//     fp16 weight tile [128 x 64] in shared memory: operand registers are built from the plane
+//     words exactly as on the decode path (1024 + sigma*v), the exact code difference
+//     q_hat - z is formed in fp16 (exact: a half-integer below 256 in magnitude), and one fp16
+//     multiply by the scale gives W_hat with a single rounding.  stmatrix writes the tiles in
+//     the swizzled layout; fence.proxy.async hands them to the tensor core;
 //   * warp 1 (one thread) issues tcgen05.mma (M = 128 weight rows, N = BN tokens, K = 16)
-//     accumulating in TMEM, and releases ring slots with tcgen05.commit;
-//   * warps 4..11 then read the fp32 accumulator with tcgen05.ld (warp w: TMEM lanes of
-//     quarter w % 4, half of the token columns each) and store y.
+//     into one of two TMEM accumulators (tiles alternate), releasing ring slots with
+//     tcgen05.commit;
+//   * warps 12..15 (one TMEM lane quarter each) read a finished accumulator with tcgen05.ld
+//     and store y while the next tile accumulates in the other one.
 //
 // fp16 (not bf16) weight tiles: with bf16 y, bf16-rounded weights exceed the 2e-3 relative
 // error budget while fp16 ones stay at the output-rounding level; both formats run at the
@@ -43,7 +46,8 @@ constexpr int kBStages = 3;     // activation-tile ring
 constexpr int kDeqWarps = 8;                   // dequantising (and epilogue) warps 4 .. 4 + kDeqWarps - 1
 constexpr int kWarpsPerTile = kDeqWarps >= 8 ? kDeqWarps / 8 : 1;  // warps sharing a 16-row tile
 constexpr int kTilesPerWarp = kDeqWarps >= 8 ? 1 : 8 / kDeqWarps;  // 16-row tiles per warp
-constexpr int kThreads = 32 * (4 + kDeqWarps);
+constexpr int kEpiWarps = 4;                    // epilogue warps 4 + kDeqWarps .. + 3 (one per TMEM lane quarter)
+constexpr int kThreads = 32 * (4 + kDeqWarps + kEpiWarps);
 constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
 
 // ---- activation conversion -----------------------------------------------------------------
@@ -86,7 +90,7 @@ struct PrefillSmem {
   static constexpr int kB = kA + kAStages * kATileBytes;
   static constexpr int kRaw = kB + kBStages * BN * 128;
   static constexpr int kBar = kRaw + kRawStages * raw_stage_bytes<R>();
-  static constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 1;
+  static constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 4;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kTotal = kTmemSlot + 16 + 1024;  // + alignment slack
 };
@@ -245,28 +249,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   uint64_t* a_empty = a_full + kAStages;
   uint64_t* b_full = a_empty + kAStages;
   uint64_t* b_empty = b_full + kBStages;
-  uint64_t* acc_full = b_empty + kBStages;
+  uint64_t* acc_full = b_empty + kBStages;   // [2]: accumulator buffer complete (tcgen05.commit)
+  uint64_t* acc_empty = acc_full + 2;        // [2]: accumulator buffer drained by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // token tiles are the fastest grid dimension: the CTAs of one weight-row block run together
-  // and share its planes through L2
-  const int rt0 = blockIdx.y * (kBM / kTileRows);
-  const int n0 = blockIdx.y * kBM;
-  const int m0 = blockIdx.x * BN;
   const int KC = P.K / kChunk;
+  // Persistent: CTA b takes tiles b, b + grid, ...; tile t = (weight-row block t / MT, token
+  // tile t % MT), token tiles fastest so that the CTAs working on one row block at a time share
+  // its planes through L2.  Two TMEM accumulators: the epilogue of tile i overlaps the MMAs of
+  // tile i + 1.
+  const int MT = (P.M + BN - 1) / BN;
+  const int tiles = MT * ((P.N + kBM - 1) / kBM);
+  const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   constexpr int kNumPlanes = planes_for_width(R);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRawStages; ++i) { mbar_init(&raw_full[i], 1); mbar_init(&raw_empty[i], kDeqWarps); }
     for (int i = 0; i < kAStages; ++i) { mbar_init(&a_full[i], 32 * kDeqWarps); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < kBStages; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], kEpiWarps); }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)BN)
+                 "r"((uint32_t)(2 * BN))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -282,21 +289,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     if (lane == 0) {
       const CUtensorMap* maps[5] = {&tm_p0, &tm_p1, &tm_p2, &tm_p3, &tm_p4};
       bool ok = true;
-      for (int kc = 0; kc < KC && ok; ++kc) {
-        const int rs = kc % kRawStages;
-        ok = mbar_wait(&raw_empty[rs], ((kc / kRawStages) & 1) ^ 1, P.err, 1);
-        if (!ok) break;
-        mbar_expect_tx(&raw_full[rs], raw_stage_bytes<R>());
-        uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
-#pragma unroll
-        for (int p = 0; p < kNumPlanes; ++p)
-          tma_load_2d(raw + raw_plane_off(p), maps[p], kc * plane_bits(p) * 64, rt0, &raw_full[rs]);
-        for (int q = 0; q < 4; ++q) {
-          const int i = kc * 4 + q, bs = i % kBStages;
-          ok = mbar_wait(&b_empty[bs], ((i / kBStages) & 1) ^ 1, P.err, 2);
+      int ic = 0, ib = 0;  // running chunk (raw ring) and 64-input slice (B ring) counts
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int t = (int)blockIdx.x + i * (int)gridDim.x;
+        const int m0 = (t % MT) * BN, rt0 = (t / MT) * (kBM / kTileRows);
+        for (int kc = 0; kc < KC && ok; ++kc, ++ic) {
+          const int rs = ic % kRawStages;
+          ok = mbar_wait(&raw_empty[rs], ((ic / kRawStages) & 1) ^ 1, P.err, 1);
           if (!ok) break;
-          mbar_expect_tx(&b_full[bs], BN * 128);
-          tma_load_2d(smem + S::kB + bs * BN * 128, &tm_x, kc * kChunk + q * kSubK, m0, &b_full[bs]);
+          mbar_expect_tx(&raw_full[rs], raw_stage_bytes<R>());
+          uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
+#pragma unroll
+          for (int p = 0; p < kNumPlanes; ++p)
+            tma_load_2d(raw + raw_plane_off(p), maps[p], kc * plane_bits(p) * 64, rt0, &raw_full[rs]);
+          for (int q = 0; q < 4; ++q, ++ib) {
+            const int bs = ib % kBStages;
+            ok = mbar_wait(&b_empty[bs], ((ib / kBStages) & 1) ^ 1, P.err, 2);
+            if (!ok) break;
+            mbar_expect_tx(&b_full[bs], BN * 128);
+            tma_load_2d(smem + S::kB + bs * BN * 128, &tm_x, kc * kChunk + q * kSubK, m0, &b_full[bs]);
+          }
         }
       }
     }
@@ -305,89 +317,108 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
       bool ok = true;
-      const int nsub = KC * 4;
-      for (int i = 0; i < nsub && ok; ++i) {
-        const int as = i % kAStages, bs = i % kBStages;
-        ok = mbar_wait(&a_full[as], (i / kAStages) & 1, P.err, 4) && mbar_wait(&b_full[bs], (i / kBStages) & 1, P.err, 8);
+      int is = 0;  // running 64-input slice count (A and B rings advance together)
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int buf = i & 1;
+        ok = mbar_wait(&acc_empty[buf], ((i >> 1) & 1) ^ 1, P.err, 128);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + S::kA + as * kATileBytes);
-        const uint32_t b_base = smem_u32(smem + S::kB + bs * BN * 128);
+        const uint32_t d = tmem_d + (uint32_t)(buf * BN);
+        for (int sub = 0; sub < KC * 4 && ok; ++sub, ++is) {
+          const int as = is % kAStages, bs = is % kBStages;
+          ok = mbar_wait(&a_full[as], (is / kAStages) & 1, P.err, 4) && mbar_wait(&b_full[bs], (is / kBStages) & 1, P.err, 8);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + S::kA + as * kATileBytes);
+          const uint32_t b_base = smem_u32(smem + S::kB + bs * BN * 128);
 #pragma unroll
-        for (int kk = 0; kk < kSubK / 16; ++kk)
-          tc_mma_f16(tmem_d, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&a_empty[as]);
-        tc_commit(&b_empty[bs]);
+          for (int kk = 0; kk < kSubK / 16; ++kk)
+            tc_mma_f16(d, sw128_desc(a_base + kk * 32), sw128_desc(b_base + kk * 32), idesc,
+                       (sub > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&a_empty[as]);
+          tc_commit(&b_empty[bs]);
+        }
+        if (ok) tc_commit(&acc_full[buf]);
       }
-      if (ok) tc_commit(acc_full);
     }
-  } else if (warp >= 4) {
-    // ---------------- dequantisation, then epilogue ----------------
+  } else if (warp >= 4 && warp < 4 + kDeqWarps) {
+    // ---------------- dequantisation ----------------
     const int wq = warp - 4;
     bool ok = true;
-    ChunkMeta<GROUP> meta;
-    load_chunk_meta<GROUP>(meta, P, 0, rt0, wq, lane);
-    for (int kc = 0; kc < KC && ok; ++kc) {
-      const int rs = kc % kRawStages;
-      if (kc > 0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
-      ok = mbar_wait(&raw_full[rs], (kc / kRawStages) & 1, P.err, 16);
-      if (!ok) break;
-      const uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
-      LaneWords L[kTilesPerWarp];
+    int ic = 0, is = 0;  // running chunk and 64-input slice counts
+    for (int i = 0; i < my_tiles && ok; ++i) {
+      const int t = (int)blockIdx.x + i * (int)gridDim.x;
+      const int rt0 = (t / MT) * (kBM / kTileRows);
+      ChunkMeta<GROUP> meta;
+      load_chunk_meta<GROUP>(meta, P, 0, rt0, wq, lane);
+      for (int kc = 0; kc < KC && ok; ++kc, ++ic) {
+        const int rs = ic % kRawStages;
+        if (kc > 0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
+        ok = mbar_wait(&raw_full[rs], (ic / kRawStages) & 1, P.err, 16);
+        if (!ok) break;
+        const uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
+        LaneWords L[kTilesPerWarp];
 #pragma unroll
-      for (int tt = 0; tt < kTilesPerWarp; ++tt)
-        lds_lane_words<R>(raw, kTilesPerWarp * (wq / kWarpsPerTile) + tt, lane, L[tt]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&raw_empty[rs]);
+        for (int tt = 0; tt < kTilesPerWarp; ++tt)
+          lds_lane_words<R>(raw, kTilesPerWarp * (wq / kWarpsPerTile) + tt, lane, L[tt]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_empty[rs]);
 #define MATQ_SUBSTAGE(Q)                                                                       \
-      if (ok) {                                                                                \
-        const int i = kc * 4 + (Q), as = i % kAStages;                                         \
-        ok = mbar_wait(&a_empty[as], ((i / kAStages) & 1) ^ 1, P.err, 32);                     \
         if (ok) {                                                                              \
-          const uint32_t a_slot = smem_u32(smem + S::kA + as * kATileBytes);                   \
-          dequant_substage<R, BN, GROUP, Q>(L, meta, wq, lane, a_slot);                        \
-          fence_proxy_async();                                                                 \
-          mbar_arrive(&a_full[as]);                                                            \
-        }                                                                                      \
-      }
-      MATQ_SUBSTAGE(0) MATQ_SUBSTAGE(1) MATQ_SUBSTAGE(2) MATQ_SUBSTAGE(3)
+          const int as = is % kAStages;                                                        \
+          ok = mbar_wait(&a_empty[as], ((is / kAStages) & 1) ^ 1, P.err, 32);                  \
+          if (ok) {                                                                            \
+            const uint32_t a_slot = smem_u32(smem + S::kA + as * kATileBytes);                 \
+            dequant_substage<R, BN, GROUP, Q>(L, meta, wq, lane, a_slot);                      \
+            fence_proxy_async();                                                               \
+            mbar_arrive(&a_full[as]);                                                          \
+          }                                                                                    \
+          ++is;                                                                                \
+        }
+        MATQ_SUBSTAGE(0) MATQ_SUBSTAGE(1) MATQ_SUBSTAGE(2) MATQ_SUBSTAGE(3)
 #undef MATQ_SUBSTAGE
+      }
     }
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 (weight rows n0 + 32*(w%4) + lane);
-    // the warp quads split the BN accumulator columns
-    if (ok) ok = mbar_wait(acc_full, 0, P.err, 64);
-    if (ok) {
+  } else if (warp >= 4 + kDeqWarps) {
+    // ---------------- epilogue ----------------
+    // warp w reads TMEM lanes 32*(w%4) .. +31 = weight rows n0 + 32*(w%4) + lane
+    const int q = warp & 3;
+    bool ok = true;
+    for (int i = 0; i < my_tiles && ok; ++i) {
+      const int buf = i & 1;
+      ok = mbar_wait(&acc_full[buf], (i >> 1) & 1, P.err, 64);
+      if (!ok) break;
       tc_fence_after();
-      const int q = warp & 3, half = wq >> 2;
-      constexpr int kQuads = (kDeqWarps / 4 < BN / 32) ? kDeqWarps / 4 : BN / 32;
-      constexpr int kChunksPerQuad = BN / 32 / kQuads;
-      const int n = n0 + 32 * q + lane;
-      const uint32_t taddr = tmem_d + ((uint32_t)(32 * q) << 16);
+      const int t = (int)blockIdx.x + i * (int)gridDim.x;
+      const int m0 = (t % MT) * BN, n = (t / MT) * kBM + 32 * q + lane;
+      const uint32_t taddr = tmem_d + (uint32_t)(buf * BN) + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
-      for (int c = half * kChunksPerQuad; half < kQuads && c < (half + 1) * kChunksPerQuad; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
         if (n < P.N) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int tok = m0 + c * 32 + i;
+          for (int k = 0; k < 32; ++k) {
+            const int tok = m0 + c * 32 + k;
             if (tok < P.M) {
               const size_t o = (size_t)tok * P.N + n;
-              if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v[i]);
-              else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v[i];
-              else reinterpret_cast<float*>(P.y)[o] += v[i];
+              if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v[k]);
+              else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v[k];
+              else reinterpret_cast<float*>(P.y)[o] += v[k];
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"((uint32_t)BN) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"((uint32_t)(2 * BN)) : "memory");
   }
 }
 
@@ -424,7 +455,12 @@ static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P
   auto kern = prefill_kernel<R, BN, GROUP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
   if (e != cudaSuccess) return e;
-  dim3 grid((P.M + BN - 1) / BN, (P.N + kBM - 1) / kBM);
+  // persistent: at most one CTA per SM (the kernel's shared memory allows no second one)
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = (long long)((P.M + BN - 1) / BN) * ((P.N + kBM - 1) / kBM);
+  dim3 grid((unsigned)(tiles < sms ? tiles : sms));
   return launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3], maps[4],
                     maps[5], P);
 }
