@@ -404,10 +404,10 @@ _KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
 NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
-    "decode": {"sha256": "ce5c2fda4d7f9c5ecb8cc359341805ebc97ebf5297651e0a555a94ad62b1cca0", "launch": "gate_up 28672x4096 r=2 M=1",
-               "bytes": 32_177_920 + 0},
-    "prefill": {"sha256": "7ef9fa1fc301969c4e1efa3dd5d4abd701a39fe5872f0a06657a8dcdb5d07be4", "launch": "gate_up 28672x4096 r=4 M=2048",
-                "bytes": 186_167_552 + 96_039_936},
+    "decode": {"sha256": "1a54fbb07df5e2053f81b536ed44241c9fb7f075ca7c28761a99abbe5a59451f", "launch": "gate_up 28672x4096 r=2 M=1",
+               "bytes": 32_177_664 + 0},
+    "prefill": {"sha256": "5ca8d9b0f2513e6bd8aa1e878e593d8f2fc2d2477dca0f2b0707811e37d549f7", "launch": "gate_up 28672x4096 r=4 M=2048",
+                "bytes": 78_527_488 + 79_799_552},
 }
 
 

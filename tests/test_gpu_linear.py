@@ -134,7 +134,7 @@ def test_decode_full_size_sampled(M, shape, group):
     dz = torch.from_numpy(z).cuda()
     planes = M.pack(dq, r_keep=8)
     rows = np.sort(np.random.default_rng(N).choice(N, 64, replace=False))
-    for Mt in (1, 4, 16):
+    for Mt in (1, 4, 8, 16):
         xb, xv = synth.activations(Mt, K, seed=0)
         dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
         for r in O.WIDTHS:

@@ -122,3 +122,48 @@ def test_mixnmatch_stack_teacher_forced(M, Mt):
     dev = np.linalg.norm(h.cpu().numpy() - h_ref) / np.linalg.norm(h_ref)
     print(f"end-to-end stack deviation (M={Mt}): {dev:.3e}")
     assert np.isfinite(dev) and dev < 5e-2
+
+
+@pytest.mark.parametrize("Mt", [1, 16, 512])
+def test_mixnmatch_stack_8b_shapes_sampled(M, Mt):
+    """The Mix'n'Match stack at the 8B FFN shapes (D = 4096, F = 14336, group 128), three layers
+    with the first widths of the seeded {2 x 11, 3 x 10, 4 x 11} permutation, gate and up served
+    by one fused call, the residual kept in fp32 by the accumulate mode.  Decode path for
+    M = 1, 16, tcgen05 prefill path for M = 512.  Every step is checked teacher-forced: the
+    projections on 512 sampled output columns, the elementwise gated product on all of them
+    (a few dozen bf16-rounded values alone can exceed the Frobenius bar by chance)."""
+    import torch
+    D, F, G, L = 4096, 14336, 128, 3
+    widths = synth.mixnmatch_widths(seed=0)[:L]
+    rng = np.random.default_rng(Mt)
+    xb, xv = synth.activations(Mt, D, seed=9)
+    h = torch.from_numpy(xv.copy()).cuda()
+    ws = M.workspace(Mt, F, 2 * F, G)
+    for l in range(L):
+        r = int(widths[l])
+        host = {nm: synth.parent_weights(N, K, G, seed=1, layer=l, proj=nm)
+                for nm, (N, K) in (("gate", (F, D)), ("up", (F, D)), ("down", (D, F)))}
+        gu = tuple(np.concatenate([host["gate"][i], host["up"][i]], axis=0) for i in range(3))
+        p_gu = M.pack(torch.from_numpy(gu[0]).cuda(), r_keep=4)      # mode A: keep 4 bits
+        p_dn = M.pack(torch.from_numpy(host["down"][0]).cuda(), r_keep=4)
+        n = M.rmsnorm(h, eps=1e-5)
+        nv = _bf16(n)
+        y_gu = M.linear(n, p_gu, 4, torch.from_numpy(gu[1].view(np.int16)).cuda(), torch.from_numpy(gu[2]).cuda(),
+                        2 * F, r, G, workspace=ws)
+        cols = np.sort(rng.choice(F, 512, replace=False))
+        for half, nm in ((0, "gate"), (1, "up")):
+            q, s, z = host[nm]
+            got = _bf16(y_gu)[:, half * F + cols]
+            check_close(got, O.linear(nv, q[cols], s[cols], z[cols], r, G), what=f"layer {l} {nm} M={Mt}")
+        a = M.silu_mul_gu(y_gu)
+        av = _bf16(a)
+        gv = _bf16(y_gu)
+        check_close(av, O.gated_product(gv[:, :F], gv[:, F:]), what=f"layer {l} silu M={Mt}")
+        h_before = h.cpu().numpy().astype(np.float64)
+        q, s, z = host["down"]
+        M.linear(a, p_dn, 4, torch.from_numpy(s.view(np.int16)).cuda(), torch.from_numpy(z).cuda(), D, r, G,
+                 y=h, y_mode=M.MATQ_OUT_F32_ACCUM, workspace=ws)
+        dcols = np.sort(rng.choice(D, 512, replace=False))
+        check_close(h.cpu().numpy()[:, dcols] - h_before[:, dcols], O.linear(av, q[dcols], s[dcols], z[dcols], r, G),
+                    what=f"layer {l} down M={Mt}")
+    assert M.workspace_status(ws) == 0
