@@ -312,10 +312,10 @@ def run_ours(args):
         s, z, N, K = meta[name]
         matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, workspace=ws)
 
-    def ffn(x, M, r, copy):
+    def ffn(x, M, r, copy, y=None):
         linear("gate_up", copy, x, r, gu_buf[M])
         matq.silu_mul_gu(gu_buf[M], out=a_buf[M])
-        linear("down", copy, a_buf[M], r, y_buf[M])
+        linear("down", copy, a_buf[M], r, y_buf[M] if y is None else y)
 
     calls = [(r, M) for r in spec["widths"] for M in batches]
 
@@ -477,20 +477,30 @@ def roofline(args, spec, linear, xs, gu_buf, stream, dev):
 
 
 def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
-    """The same step through the public calls, with each call's activations copied in from
-    pinned host memory and its output copied back, inside the timed region."""
+    """The same step through the public calls, with the step's activations copied in from
+    pinned host memory (one copy of all of them) and its outputs copied back (one copy of all
+    of them), inside the timed region."""
     import torch
-    host_x = {M: xs[M].cpu().pin_memory() for M in xs}
-    host_y = {M: torch.empty_like(y_buf[M], device="cpu").pin_memory() for M in y_buf}
-    dev_x = {M: torch.empty_like(xs[M]) for M in xs}
-    h2d = sum(host_x[M].numel() * 2 for (_, M) in calls)
-    d2h = sum(host_y[M].numel() * 2 for (_, M) in calls)
+    # the step's inputs and outputs, one slice per FFN call, in one pinned buffer each way
+    offs, o = [], 0
+    for (_, M) in calls:
+        offs.append(o)
+        o += M
+    rows = o
+    host_x = torch.empty((rows, D_MODEL), dtype=torch.bfloat16).pin_memory()
+    for (_, M), off in zip(calls, offs):
+        host_x[off:off + M].copy_(xs[M].cpu())
+    host_y = torch.empty((rows, D_MODEL), dtype=torch.bfloat16).pin_memory()
+    dev_x = torch.empty((rows, D_MODEL), dtype=torch.bfloat16, device=dev)
+    dev_y = torch.empty((rows, D_MODEL), dtype=torch.bfloat16, device=dev)
+    h2d = host_x.numel() * 2
+    d2h = host_y.numel() * 2
 
     def step(base=0):
-        for i, (r, M) in enumerate(calls):
-            dev_x[M].copy_(host_x[M], non_blocking=True)
-            ffn(dev_x[M], M, r, (base + i) % args.copies)
-            host_y[M].copy_(y_buf[M], non_blocking=True)
+        dev_x.copy_(host_x, non_blocking=True)
+        for i, ((r, M), off) in enumerate(zip(calls, offs)):
+            ffn(dev_x[off:off + M], M, r, (base + i) % args.copies, y=dev_y[off:off + M])
+        host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(max(1, args.warmup)):

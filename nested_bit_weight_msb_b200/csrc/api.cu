@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <atomic>
+
 #include "../../include/matq.h"
 #include "common.cuh"
 #include "internal.h"
@@ -50,6 +52,29 @@ size_t packed_bytes(int N, int K, int r_keep) {
 }  // namespace
 
 namespace matq {
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// SM count per device, queried once (the attribute cannot change during the process).
+int sm_count(int dev) {
+  static std::atomic<int> cache[64];
+  if (dev < 0 || dev >= 64) {
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 // Status helpers for the other translation units of the C ABI.
 int record_cuda_error(cudaError_t e) { return cuda_status(e); }
 int check_sm100_device() { return check_device(); }

@@ -40,6 +40,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "operands.cuh"
@@ -612,8 +614,15 @@ static cudaError_t launch_decode_t(const uint8_t* planes, const PlaneGeom& g, De
   const long long ctas = (long long)sms * CPS;
   P.C = (int)(P.I < ctas ? P.I : ctas);
   auto kern = decode_kernel<R, NT, GROUP, CPS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem);
-  if (e != cudaSuccess) return e;
+  // the shared-memory attribute is set once per device for this kernel
+  static std::atomic<unsigned long long> attr_set{0};
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (dev >= 64 || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit, std::memory_order_relaxed);
+  }
   return launch_pdl(kern, dim3(P.C), dim3(Lt::kThreads), (size_t)Lt::kSmem, s, maps[0], maps[1], maps[2], maps[3],
                     maps[4], P);
 }
@@ -635,9 +644,7 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
                           cudaStream_t s) {
   const int NT = (M <= 8) ? 1 : 2;
   uint8_t* ws = (uint8_t*)workspace;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = sm_count(current_device());
   if (sms > kMaxSMs) sms = kMaxSMs;
   DecodeParams P;
   P.N = g.N;

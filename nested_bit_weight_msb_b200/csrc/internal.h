@@ -27,6 +27,11 @@ cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, c
 cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s);
 cudaError_t launch_silu_mul_gu(const void* gu, int M, int F, void* out, cudaStream_t s);
 
+// Host-side per-device caches (api.cu): the SM count of the current device, and the device
+// index with which a launcher records that a kernel's shared-memory attribute is set.
+int current_device();
+int sm_count(int dev);
+
 // C-ABI status helpers (api.cu): record a failed CUDA call as the thread's last CUDA error and
 // return MATQ_ECUDA; check that the current device is an sm_100 part.
 int record_cuda_error(cudaError_t e);

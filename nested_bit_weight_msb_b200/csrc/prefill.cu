@@ -31,6 +31,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 #include "operands.cuh"
@@ -453,12 +455,17 @@ template <int R, int BN, int GROUP>
 static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
   using S = PrefillSmem<R, BN>;
   auto kern = prefill_kernel<R, BN, GROUP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
-  if (e != cudaSuccess) return e;
+  // the shared-memory attribute is set once per device for this kernel
+  static std::atomic<unsigned long long> attr_set{0};
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (dev >= 64 || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit, std::memory_order_relaxed);
+  }
   // persistent: at most one CTA per SM (the kernel's shared memory allows no second one)
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count(dev);
   const long long tiles = (long long)((P.M + BN - 1) / BN) * ((P.N + kBM - 1) / kBM);
   dim3 grid((unsigned)(tiles < sms ? tiles : sms));
   return launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3], maps[4],
