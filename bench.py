@@ -67,6 +67,14 @@ def workload_spec(name):
     return dict(widths=(3, 4, 8), batches=(2048,), outlier=0.01, unit="TFLOP/s")
 
 
+def workload_config(args, spec, world):
+    """The workload both arms report (the reference arm adds where it runs)."""
+    return {"workload": args.workload,
+            "shapes": "gate+up fused [28672,4096] (two [14336,4096] stacked), down [4096,14336], group 128",
+            "widths": list(spec["widths"]), "batches": list(spec["batches"]),
+            "parallelism": f"replicas x{world}"}
+
+
 def linear_bytes(M, N, K, r, group=GROUP):
     G = K // group
     return N * K * r // 8 + N * G * 3 + M * K * 2 + M * N * 2
@@ -262,7 +270,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": v, "unit": spec["unit"], "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_units / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "device": "cpu"},
+        "config": dict(workload_config(args, spec, world), device="host cores (fp64 oracle)"),
         "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"], "value": v,
                          "unit": spec["unit"]},
         "e2e": {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -363,11 +371,9 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16-operands/f32-acc (bf16 in/out)", "data": "synthetic",
-            "config": {"workload": args.workload,
-                       "shapes": "gate+up fused [28672,4096] (two [14336,4096] stacked), down [4096,14336], group 128",
-                       "widths": list(spec["widths"]), "batches": list(batches),
-                       "l2": f"rotating {args.copies} device copies of the packed layer (> L2)",
-                       "parallelism": f"replicas x{world}", "timing": "CUDA graph replay, CUDA events"},
+            "config": dict(workload_config(args, spec, world),
+                           l2=f"rotating {args.copies} device copies of the packed layer (> L2)",
+                           timing="CUDA graph replay, CUDA events"),
             "roofline": rl,
             "e2e": e2e,
             # per FFN: fused gate+up and down (one kernel each on the decode path, conversion +
