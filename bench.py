@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
     ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--case", choices=["decode", "prefill", "pack"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
     ap.add_argument("--m", type=int, default=1)
@@ -527,9 +527,44 @@ def end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world):
             "ms_per_step": ms}
 
 
+def run_pack_case(args):
+    """The one-time int8 -> plane-layout pack of every 8B and 9B FFN matrix (all planes,
+    r_keep = 8), timed with CUDA events over 20 back-to-back packs each (inputs > L2):
+    GB/s of its N*K bytes read + N*K bytes written."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq
+    torch.cuda.set_device(0)
+    rng = np.random.default_rng(0)
+    out = {}
+    for name, (N, K) in (("8b gate/up", (14336, 4096)), ("8b down", (4096, 14336)),
+                         ("9b gate/up", (14336, 3584)), ("9b down", (3584, 14336))):
+        codes = [torch.from_numpy(rng.integers(0, 256, (N, K), dtype=np.uint8)).cuda() for _ in range(3)]
+        planes = torch.empty(matq.matq_packed_bytes(N, K, 8), dtype=torch.uint8, device="cuda")
+        stream = torch.cuda.current_stream()
+        for i in range(3):
+            matq.check(matq.matq_pack(codes[i].data_ptr(), N, K, 8, planes.data_ptr(), planes.numel(),
+                                      stream.cuda_stream), "matq_pack")
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n = 20
+        e0.record()
+        for i in range(n):
+            matq.check(matq.matq_pack(codes[i % 3].data_ptr(), N, K, 8, planes.data_ptr(), planes.numel(),
+                                      stream.cuda_stream), "matq_pack")
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / n * 1e3
+        out[name] = {"us": round(us, 2), "GB/s": round(2 * N * K / us / 1e3, 1)}
+    print(json.dumps({"case": "pack", "r_keep": 8, "results": out}))
+    return 0
+
+
 def run_case(args):
     """A few single calls of the fused gate+up projection (28672 x 4096, group 128) at width r
-    and batch m, rotating through device copies of the pack (> L2); used for ncu captures."""
+    and batch m, rotating through device copies of the pack (> L2); used for ncu captures.
+    `--case pack` times the one-time pack instead."""
+    if args.case == "pack":
+        return run_pack_case(args)
     import torch
     from nested_bit_weight_msb_b200 import matq, synth
     torch.cuda.set_device(0)
