@@ -3,9 +3,12 @@
 Workload (default, ``--workload ffn8b_decode``): the Llama-3.1-8B-shaped FFN at decode
 batch sizes.  One step runs, for every width r in {2, 3, 4, 6, 8} and every batch
 M in {1, 4, 16}, one FFN forward through the sliced linears:
-    gu   = x . [W_gate; W_up]_r^T   [M, 28672]   (one matq_linear call: gate and up share x)
-    a    = silu(gu[:, :14336]) * gu[:, 14336:]  (matq_silu_mul_gu)
+    a    = silu(x . W_gate,r^T) * (x . W_up,r^T)   [M, 14336]   (ONE matq_linear call over the
+           row-interleaved [gate; up] pack, MATQ_OUT_SILU_GATED: the gated product is formed
+           in the epilogue from the fp32 results)
     y    = a . W_down,r^T           [M, 4096]
+(on the prefill workload the gate+up call writes both halves, [M, 28672], and matq_silu_mul_gu
+forms the product: there the epilogue arithmetic would compete with the dequantising warps)
 with group-128 parent codes of N(0, 0.02) weights (synthetic, seeded) and N(0, 1) bf16
 activations.  ``value`` = algorithmic bytes of the sliced linears (planes of width r,
 fp16 scales, uint8 zeros, x, y) over the device time of the step -> GB/s.
@@ -69,19 +72,32 @@ def workload_spec(name):
 
 def workload_config(args, spec, world):
     """The workload both arms report (the reference arm adds where it runs)."""
+    gu = ("gated product in the epilogue" if gated_epilogue(spec)
+          else "both halves written, gated product by matq_silu_mul_gu")
     return {"workload": args.workload,
-            "shapes": "gate+up fused [28672,4096] (two [14336,4096] stacked), down [4096,14336], group 128",
+            "shapes": f"gate+up [28672,4096] (two [14336,4096] row-interleaved, {gu}), down [4096,14336], group 128",
             "widths": list(spec["widths"]), "batches": list(spec["batches"]),
             "parallelism": f"replicas x{world}"}
 
 
-def linear_bytes(M, N, K, r, group=GROUP):
+def linear_bytes(M, N, K, r, group=GROUP, out_cols=None):
     G = K // group
-    return N * K * r // 8 + N * G * 3 + M * K * 2 + M * N * 2
+    return N * K * r // 8 + N * G * 3 + M * K * 2 + M * (N if out_cols is None else out_cols) * 2
 
 
-# the sliced-linear calls of one FFN: fused gate+up, then down
+# the sliced-linear calls of one FFN: gate+up over the row-interleaved pack, then down
 FFN_CALLS = (("gate_up", (2 * D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))
+
+
+def gated_epilogue(spec):
+    """The gated product is fused into the gate+up call on the decode workload only."""
+    return spec["unit"] == "GB/s"
+
+
+def out_cols(spec, name):
+    if name == "gate_up":
+        return D_FF if gated_epilogue(spec) else 2 * D_FF
+    return D_MODEL
 
 
 def step_units(spec):
@@ -89,8 +105,8 @@ def step_units(spec):
     b = f = 0
     for r in spec["widths"]:
         for M in spec["batches"]:
-            for _, (N, K) in FFN_CALLS:
-                b += linear_bytes(M, N, K, r)
+            for name, (N, K) in FFN_CALLS:
+                b += linear_bytes(M, N, K, r, out_cols=out_cols(spec, name))
                 f += 2 * M * N * K
     return b, f
 
@@ -238,10 +254,18 @@ def host_weights():
             for name, (N, K) in (("gate", (D_FF, D_MODEL)), ("up", (D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))}
 
 
+def interleave_rows(a, b):
+    out = np.empty((2 * a.shape[0],) + a.shape[1:], dtype=a.dtype)
+    out[0::2] = a
+    out[1::2] = b
+    return out
+
+
 def fused_weights(w):
-    """gate and up read the same x: their codes, scales and zero points are stacked along N
-    into one [2F, D] matrix served by one call."""
-    gu = tuple(np.concatenate([w["gate"][i], w["up"][i]], axis=0) for i in range(3))
+    """gate and up read the same x: their codes, scales and zero points are interleaved by
+    row (2i: gate row i, 2i + 1: up row i) into one [2F, D] matrix served by one call whose
+    epilogue forms silu(gate) * up."""
+    gu = tuple(interleave_rows(w["gate"][i], w["up"][i]) for i in range(3))
     return {"gate_up": gu, "down": w["down"]}
 
 
@@ -312,17 +336,22 @@ def run_ours(args):
     Mmax = max(batches)
     ws = torch.zeros(max(matq.workspace_bytes(Mmax, K, N, GROUP) for _, (N, K) in FFN_CALLS),
                      dtype=torch.uint8, device=dev)
-    gu_buf = {M: torch.empty((M, 2 * D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
     a_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
+    gated = gated_epilogue(spec)
+    gu_buf = {M: torch.empty((M, out_cols(spec, "gate_up")), dtype=torch.bfloat16, device=dev) for M in batches}
     y_buf = {M: torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev) for M in batches}
 
     def linear(name, copy, x, r, out):
         s, z, N, K = meta[name]
-        matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, workspace=ws)
+        mode = matq.MATQ_OUT_SILU_GATED if (name == "gate_up" and gated) else matq.MATQ_OUT_BF16
+        matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, y_mode=mode, workspace=ws)
 
     def ffn(x, M, r, copy, y=None):
-        linear("gate_up", copy, x, r, gu_buf[M])
-        matq.silu_mul_gu(gu_buf[M], out=a_buf[M])
+        if gated:
+            linear("gate_up", copy, x, r, a_buf[M])
+        else:
+            linear("gate_up", copy, x, r, gu_buf[M])
+            matq.silu_mul_gu(gu_buf[M], out=a_buf[M])
         linear("down", copy, a_buf[M], r, y_buf[M] if y is None else y)
 
     calls = [(r, M) for r in spec["widths"] for M in batches]
@@ -376,9 +405,9 @@ def run_ours(args):
                            timing="CUDA graph replay, CUDA events"),
             "roofline": rl,
             "e2e": e2e,
-            # per FFN: fused gate+up and down (one kernel each on the decode path, conversion +
-            # GEMM on the prefill path) and the SiLU-gated product
-            "gpu_launches": args.steps * len(calls) * (len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2) + 1),
+            # per FFN: gated gate+up and down, one kernel each on the decode path; on the prefill
+            # path activation conversion + GEMM each, and the gated product
+            "gpu_launches": args.steps * len(calls) * (len(FFN_CALLS) if gated else 2 * len(FFN_CALLS) + 1),
             "clocks": clk.summary(),
             "peaks_source": peaks.get("_source"),
         }
@@ -464,9 +493,9 @@ def roofline(args, spec, linear, xs, gu_buf, stream, dev):
     del g
     avg_ms = float(np.median(reps))
     N = 2 * D_FF
-    launch = f"gate_up {N}x{D_MODEL} r={r} M={M}"
+    launch = f"gate_up {'gated ' if gated_epilogue(spec) else ''}{N}x{D_MODEL} r={r} M={M}"
     if spec["unit"] == "GB/s":
-        units = linear_bytes(M, N, D_MODEL, r)
+        units = linear_bytes(M, N, D_MODEL, r, out_cols=out_cols(spec, "gate_up"))
         ach = units / (avg_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -560,8 +589,10 @@ def run_pack_case(args):
 
 
 def run_case(args):
-    """A few single calls of the fused gate+up projection (28672 x 4096, group 128) at width r
-    and batch m, rotating through device copies of the pack (> L2); used for ncu captures.
+    """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128;
+    gated-product epilogue for --case decode, both halves written for --case prefill, as in
+    the workloads) at width r and batch m, rotating through device copies of the pack (> L2);
+    used for ncu captures.
     `--case pack` times the one-time pack instead."""
     if args.case == "pack":
         return run_pack_case(args)
@@ -577,9 +608,11 @@ def run_case(args):
     xb, _ = synth.activations(args.m, D_MODEL, seed=0, outlier_frac=0.01 if args.case == "prefill" else 0.0)
     dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
     ws = matq.workspace(args.m, D_MODEL, N, GROUP)
-    y = torch.empty((args.m, N), dtype=torch.bfloat16, device="cuda")
+    gated = args.case == "decode"
+    y = torch.empty((args.m, N // 2 if gated else N), dtype=torch.bfloat16, device="cuda")
+    mode = matq.MATQ_OUT_SILU_GATED if gated else matq.MATQ_OUT_BF16
     for i in range(args.calls):
-        matq.linear(dx, packs[i % len(packs)], 8, ds, dz, N, args.r, GROUP, y=y, workspace=ws)
+        matq.linear(dx, packs[i % len(packs)], 8, ds, dz, N, args.r, GROUP, y=y, y_mode=mode, workspace=ws)
     torch.cuda.synchronize()
     assert matq.workspace_status(ws) == 0
     print(json.dumps({"case": args.case, "r": args.r, "m": args.m, "calls": args.calls, "ok": True}))

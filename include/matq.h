@@ -87,6 +87,7 @@ extern "C" {
 #define MATQ_OUT_BF16       0   /* y [M, N] bf16 = x . W_hat^T                             */
 #define MATQ_OUT_F32        1   /* y [M, N] fp32 = x . W_hat^T                             */
 #define MATQ_OUT_F32_ACCUM  2   /* y [M, N] fp32 += x . W_hat^T (fused residual add)       */
+#define MATQ_OUT_SILU_GATED 3   /* y [M, N/2] bf16 = silu(gate) * up, rows paired (below)  */
 
 /* Library version (major*10000 + minor*100 + patch). */
 int matq_version(void);
@@ -154,7 +155,11 @@ int matq_workspace_status(const void* workspace, int* status_out);
  *   x        [M, K] bf16, row-major, device.  Read only.
  *   planes   pack with r_keep >= r.  Read only; exactly the planes of width r are read.
  *   scales   [N, K/group] fp16 (raw bits), row-major.  zeros [N, K/group] uint8.
- *   y        [M, N] row-major, dtype by y_mode (MATQ_OUT_*).  MATQ_OUT_F32_ACCUM adds the
+ *   y        [M, N] row-major, dtype by y_mode (MATQ_OUT_*).  MATQ_OUT_SILU_GATED: N even and
+ *            the weight rows interleave the gate and up projections of an FFN (row 2i: gate
+ *            row i, row 2i + 1: up row i); y is [M, N/2] bf16 with y[m, i] =
+ *            bf16( silu(g) * u ), g and u the fp32 results of rows 2i and 2i + 1 (the gated
+ *            product fused into the epilogue; silu(t) = t / (1 + exp(-t))).  MATQ_OUT_F32_ACCUM adds the
  *            product to the fp32 values already in y.
  *   workspace device scratch of >= matq_linear_workspace(M, K, N, group) bytes, owned by
  *            the caller, header zero-filled once (see matq_workspace_init).

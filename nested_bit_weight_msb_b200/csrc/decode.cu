@@ -333,13 +333,33 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
             else reinterpret_cast<float*>(P.y)[o] += v;
           }
         };
+        // Four values of one (row tile j, token tile nt) fragment; the whole warp calls this.
+        // Gated mode: even rows (gate) take the odd row below (up) from the lane 4 higher and
+        // write silu(gate) * up at column row / 2 of y [M, N/2].
+        auto store4 = [&](int j, int nt, float v0, float v1, float v2, float v3) {
+          if (P.y_mode == 3) {
+            const float vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float u = __shfl_down_sync(0xffffffffu, vv[i], 4);
+              const int row = (rg * RG + rs * RPW + j) * 16 + gid + 8 * (i >> 1);
+              const int tok = nt * 8 + 2 * tg + (i & 1);
+              if ((gid & 1) == 0 && row < P.N && tok < P.M)
+                reinterpret_cast<__nv_bfloat16*>(P.y)[(size_t)tok * (P.N >> 1) + (row >> 1)] =
+                    __float2bfloat16_rn(__fdividef(vv[i], 1.0f + __expf(-vv[i])) * u);
+            }
+            return;
+          }
+          store_y(j, nt, 0, v0);
+          store_y(j, nt, 1, v1);
+          store_y(j, nt, 2, v2);
+          store_y(j, nt, 3, v3);
+        };
         if (whole) {
 #pragma unroll
           for (int j = 0; j < RPW; ++j)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) store_y(j, nt, i, yacc[j][nt][i]);
+            for (int nt = 0; nt < NT; ++nt) store4(j, nt, yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
         } else if (ok) {
           // Split row group: its first contributor c_first works on it last (its items end
           // c_first's range and start everybody else's), so c_first combines; the others
@@ -414,12 +434,8 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
 #pragma unroll
             for (int j = 0; j < RPW; ++j)
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                store_y(j, nt, 0, acc[j * NT + nt].x);
-                store_y(j, nt, 1, acc[j * NT + nt].y);
-                store_y(j, nt, 2, acc[j * NT + nt].z);
-                store_y(j, nt, 3, acc[j * NT + nt].w);
-              }
+              for (int nt = 0; nt < NT; ++nt)
+                store4(j, nt, acc[j * NT + nt].x, acc[j * NT + nt].y, acc[j * NT + nt].z, acc[j * NT + nt].w);
           }
         }
       }

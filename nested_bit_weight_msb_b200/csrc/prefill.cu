@@ -398,7 +398,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
-        if (n < P.N) {
+        if (P.y_mode == 3) {
+          // gated mode: even rows (gate) take the odd row below (up) from the next lane and
+          // write silu(gate) * up at column n / 2 of y [M, N/2]
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float u = __shfl_down_sync(0xffffffffu, v[k], 1);
+            const int tok = m0 + c * 32 + k;
+            if ((lane & 1) == 0 && n < P.N && tok < P.M)
+              reinterpret_cast<__nv_bfloat16*>(P.y)[(size_t)tok * (P.N >> 1) + (n >> 1)] =
+                  __float2bfloat16_rn(__fdividef(v[k], 1.0f + __expf(-v[k])) * u);
+          }
+        } else if (n < P.N) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
             const int tok = m0 + c * 32 + k;

@@ -74,7 +74,8 @@ extern "C" int matq_linear_noalloc(const void* x, int M, int K, const void* plan
     return MATQ_EINVAL_SHAPE;
   if (M <= kDecodeMaxM && (long long)N > max_decode_rows()) return MATQ_EINVAL_SHAPE;
   if (group != 64 && group != 128) return MATQ_EINVAL_GROUP;
-  if (y_mode < MATQ_OUT_BF16 || y_mode > MATQ_OUT_F32_ACCUM) return MATQ_EDTYPE;
+  if (y_mode < MATQ_OUT_BF16 || y_mode > MATQ_OUT_SILU_GATED) return MATQ_EDTYPE;
+  if (y_mode == MATQ_OUT_SILU_GATED && (N & 1)) return MATQ_EINVAL_SHAPE;
   if (!x || !planes || !scales || !zeros || !y) return MATQ_ENULL;
   if (!aligned16(x) || !aligned16(planes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||
       ((uintptr_t)status_out & 3u))

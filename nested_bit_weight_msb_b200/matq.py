@@ -39,6 +39,7 @@ MATQ_ESCRATCH = -11
 MATQ_OUT_BF16 = 0
 MATQ_OUT_F32 = 1
 MATQ_OUT_F32_ACCUM = 2
+MATQ_OUT_SILU_GATED = 3
 
 WIDTHS = (2, 3, 4, 6, 8)
 DECODE_MAX_M = 16
@@ -162,8 +163,9 @@ def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=
     torch = _torch()
     M, K = x.shape
     if y is None:
-        dt = torch.bfloat16 if y_mode == MATQ_OUT_BF16 else torch.float32
-        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, N), dtype=dt, device=x.device)
+        dt = torch.bfloat16 if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else torch.float32
+        cols = N // 2 if y_mode == MATQ_OUT_SILU_GATED else N
+        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, cols), dtype=dt, device=x.device)
     if workspace is None:
         workspace = torch.zeros(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
     check(matq_linear(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
@@ -179,8 +181,9 @@ def linear_noalloc(x, planes, r_keep: int, scales, zeros, N: int, r: int, group:
     torch = _torch()
     M, K = x.shape
     if y is None:
-        dt = torch.bfloat16 if y_mode == MATQ_OUT_BF16 else torch.float32
-        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, N), dtype=dt, device=x.device)
+        dt = torch.bfloat16 if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else torch.float32
+        cols = N // 2 if y_mode == MATQ_OUT_SILU_GATED else N
+        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, cols), dtype=dt, device=x.device)
     sp = _ptr(status) if status is not None else None
     check(matq_linear_noalloc(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
                               _ptr(y), y_mode, sp, _stream_ptr(stream)), "matq_linear_noalloc")

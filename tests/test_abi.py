@@ -99,7 +99,9 @@ def test_linear_rejects(M):
     assert call(K=1000) == M.MATQ_EINVAL_SHAPE
     assert call(N=0) == M.MATQ_EINVAL_SHAPE
     assert call(group=32) == M.MATQ_EINVAL_GROUP
-    assert call(y_mode=3) == M.MATQ_EDTYPE
+    assert call(y_mode=4) == M.MATQ_EDTYPE
+    assert call(y_mode=-1) == M.MATQ_EDTYPE
+    assert call(y_mode=M.MATQ_OUT_SILU_GATED, N=63) == M.MATQ_EINVAL_SHAPE
     assert call(x=None) == M.MATQ_ENULL
     assert call(zeros=FAKE + 4) == M.MATQ_EALIGN
     assert call(ws_bytes=16) == M.MATQ_ESIZE

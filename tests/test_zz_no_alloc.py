@@ -29,7 +29,8 @@ def test_noalloc_rejects_before_any_launch(M):
     assert _call(M, r=8, r_keep=4) == M.MATQ_ETRUNC
     assert _call(M, K=1000) == M.MATQ_EINVAL_SHAPE
     assert _call(M, group=32) == M.MATQ_EINVAL_GROUP
-    assert _call(M, y_mode=3) == M.MATQ_EDTYPE
+    assert _call(M, y_mode=4) == M.MATQ_EDTYPE
+    assert _call(M, y_mode=M.MATQ_OUT_SILU_GATED, N=63) == M.MATQ_EINVAL_SHAPE
     assert _call(M, x=None) == M.MATQ_ENULL
     assert _call(M, y=FAKE + 8) == M.MATQ_EALIGN
     assert _call(M, status=FAKE + 2) == M.MATQ_EALIGN
