@@ -439,10 +439,10 @@ _KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
 NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
-    "decode": {"sha256": "1a54fbb07df5e2053f81b536ed44241c9fb7f075ca7c28761a99abbe5a59451f", "launch": "gate_up 28672x4096 r=2 M=1",
-               "bytes": 32_177_664 + 0},
-    "prefill": {"sha256": "5ca8d9b0f2513e6bd8aa1e878e593d8f2fc2d2477dca0f2b0707811e37d549f7", "launch": "gate_up 28672x4096 r=4 M=2048",
-                "bytes": 78_527_488 + 79_799_552},
+    "decode": {"sha256": "0532170b3041f920007ae78a117291f110bc4db70afbe0a4056be508aefd1756", "launch": "gate_up gated 28672x4096 r=2 M=1",
+               "bytes": 32_189_952 + 0},
+    "prefill": {"sha256": "e65082c36fd9bc05759950ee33e9ec7141f7a1b6b9df61b7c7cceafd9d884e25", "launch": "gate_up 28672x4096 r=4 M=2048",
+                "bytes": 78_459_904 + 79_054_848},
 }
 
 
