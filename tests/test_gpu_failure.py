@@ -1,0 +1,104 @@
+"""Failure detection and output bounds on the GPU, without faulting it.
+
+* A workspace whose header was not zero-filled (a caller error) leaves the split-row-group
+  counters wrong: the combining warps' bounded waits run out (about a second), record their
+  error code in the header, skip the combine and return; the host reads the status, and after
+  matq_workspace_init the same workspace gives correct results again.
+* Canary-padded outputs: nothing is written past the [M, N] (or [M, N/2]) output, for ragged
+  rows and token counts on both paths and in every output mode.
+"""
+
+import numpy as np
+import pytest
+
+import oracle as O
+from helpers import check_close, problem, to_device
+
+pytestmark = pytest.mark.gpu
+
+COMBINE_TIMEOUT = 128  # device status code of a split-row-group combine whose wait ran out
+
+
+@pytest.fixture(scope="module")
+def M():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from nested_bit_weight_msb_b200 import matq
+    return matq
+
+
+def test_uninitialised_workspace_is_detected_and_recoverable(M):
+    import torch
+    Mt, N, K, G, r = 1, 4096, 4096, 128, 2   # 256 items on 148 CTAs: row groups are split
+    q, s, z, xb, xv = problem(Mt, N, K, G, seed=21)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    ws = M.workspace(Mt, K, N, G)
+    # corrupt the split-row-group counters (the header after the two status words)
+    ws[256:256 + 65536 * 4].view(torch.int32).fill_(-(1 << 30))
+    M.linear(dx, planes, 8, ds, dz, N, r, G, workspace=ws)
+    torch.cuda.synchronize()
+    st = M.workspace_status(ws)
+    assert st & COMBINE_TIMEOUT, f"status {st}"
+    # the context is usable and the workspace recovers after re-initialisation
+    M.check(M.matq_workspace_init(ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream),
+            "matq_workspace_init")
+    y = M.linear(dx, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32, workspace=ws)
+    torch.cuda.synchronize()
+    assert M.workspace_status(ws) == 0
+    rows = np.arange(0, N, 7)
+    check_close(y.cpu().numpy()[:, rows], O.linear(xv, q[rows], s[rows], z[rows], r, G), what="after recovery")
+
+
+def _canary(torch, n, dtype):
+    buf = torch.empty(n + 4096, dtype=dtype, device="cuda")
+    buf.view(torch.uint8).fill_(0xA5)
+    return buf
+
+
+@pytest.mark.parametrize("Mt,N,K,mode", [(1, 1000, 1024, 0), (7, 333, 512, 1), (16, 1000, 768, 2),
+                                         (5, 1002, 512, 3), (17, 1000, 512, 0), (129, 130, 512, 1),
+                                         (40, 1002, 256, 3), (300, 250, 1024, 2)])
+def test_outputs_stay_in_bounds(M, Mt, N, K, mode):
+    import torch
+    G, r = 128, 4
+    q, s, z, xb, xv = problem(Mt, N, K, G, seed=Mt + N)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    cols = N // 2 if mode == M.MATQ_OUT_SILU_GATED else N
+    dt = torch.bfloat16 if mode in (M.MATQ_OUT_BF16, M.MATQ_OUT_SILU_GATED) else torch.float32
+    buf = _canary(torch, Mt * cols, dt)
+    y = buf[:Mt * cols].view(Mt, cols)
+    if mode == M.MATQ_OUT_F32_ACCUM:
+        y.zero_()
+    M.linear(dx, planes, 8, ds, dz, N, r, G, y=y, y_mode=mode)
+    torch.cuda.synchronize()
+    tail = buf[Mt * cols:].view(torch.uint8)
+    assert bool((tail == 0xA5).all()), "write past the output"
+    ref = O.linear(xv, q, s, z, r, G)
+    if mode == M.MATQ_OUT_SILU_GATED:
+        ref = O.gated_product(ref[:, 0::2], ref[:, 1::2])
+        got = y.float().cpu().numpy()
+        err = np.abs(got - ref)
+        assert np.all(err <= 1e-2 * (np.abs(ref) + 1)), "gated output"
+    else:
+        check_close(y.float().cpu().numpy(), ref, what=f"mode {mode}")
+
+
+def test_glue_outputs_stay_in_bounds(M):
+    import torch
+    Mt, F = 3, 1001
+    g = torch.randn(Mt, F, device="cuda").to(torch.bfloat16)
+    u = torch.randn(Mt, F, device="cuda").to(torch.bfloat16)
+    buf = _canary(torch, Mt * F, torch.bfloat16)
+    M.silu_mul(g, u, out=buf[:Mt * F].view(Mt, F))
+    gu = torch.randn(Mt, 2 * F, device="cuda").to(torch.bfloat16)
+    buf2 = _canary(torch, Mt * F, torch.bfloat16)
+    M.silu_mul_gu(gu, out=buf2[:Mt * F].view(Mt, F))
+    h = torch.randn(Mt, F, device="cuda")
+    buf3 = _canary(torch, Mt * F, torch.bfloat16)
+    M.rmsnorm(h, out=buf3[:Mt * F].view(Mt, F))
+    torch.cuda.synchronize()
+    for b in (buf, buf2, buf3):
+        assert bool((b[Mt * F:].view(torch.uint8) == 0xA5).all()), "write past the output"

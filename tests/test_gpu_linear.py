@@ -48,7 +48,7 @@ def test_single_linear_1024(M, r):
 
 
 @pytest.mark.parametrize("group", [64, 128])
-@pytest.mark.parametrize("Mt", [1, 2, 3, 5, 8, 9, 12, 16])
+@pytest.mark.parametrize("Mt", [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16])
 def test_decode_small_sweep(M, Mt, group):
     """Several row tiles with a ragged last tile, several chunks, every width."""
     N, K = 83, 768
@@ -150,8 +150,8 @@ def _device_status(M, ws, Mt, K, N, group):
     return M.workspace_status(ws)
 
 
-@pytest.mark.parametrize("Mt,N,K,group", [(17, 128, 256, 128), (64, 200, 512, 64), (100, 384, 768, 128),
-                                          (129, 130, 512, 64), (300, 256, 1024, 128)])
+@pytest.mark.parametrize("Mt,N,K,group", [(17, 128, 256, 128), (31, 300, 512, 128), (64, 200, 512, 64),
+                                          (100, 384, 768, 128), (129, 130, 512, 64), (300, 256, 1024, 128)])
 def test_prefill_small(M, Mt, N, K, group):
     """Tiles of every token-tile size (64, 128, 256), ragged tokens and rows, both groups."""
     import torch
