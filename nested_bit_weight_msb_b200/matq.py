@@ -109,32 +109,53 @@ def _ptr(t) -> int:
     return int(t.data_ptr())
 
 
+def _dev(t, name: str, dtypes, what: str):
+    """Pointer of a CUDA tensor after the checks the C ABI cannot make itself: the memory is
+    on the GPU, contiguous, of an accepted element type.  (A host pointer or a strided view
+    would be read as garbage, or fault.)"""
+    if not t.is_cuda:
+        raise ValueError(f"{what}: {name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: {name} must be contiguous")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{what}: {name} has dtype {t.dtype}, expected one of {dtypes}")
+    return int(t.data_ptr())
+
+
+def _dt(*names):
+    torch = _torch()
+    return tuple(getattr(torch, n) for n in names)
+
+
 def pack(codes, r_keep: int = 8, stream=None):
     """Pack [N, K] uint8 codes (CUDA tensor) into a uint8 plane buffer (CUDA tensor)."""
     torch = _torch()
     N, K = codes.shape
+    pc = _dev(codes, "codes", _dt("uint8"), "pack")
     nbytes = matq_packed_bytes(N, K, r_keep)
     if nbytes == 0:
         check(MATQ_EINVAL_SHAPE if r_keep in WIDTHS else MATQ_EINVAL_R, "matq_packed_bytes")
     planes = torch.empty(nbytes, dtype=torch.uint8, device=codes.device)
-    check(matq_pack(_ptr(codes), N, K, r_keep, _ptr(planes), nbytes, _stream_ptr(stream)), "matq_pack")
+    check(matq_pack(pc, N, K, r_keep, _ptr(planes), nbytes, _stream_ptr(stream)), "matq_pack")
     return planes
 
 
 def slice_prefix(planes, N: int, K: int, r_keep: int, r: int, stream=None):
     """Prefixes p = q >> (8 - r) as a [N, K] uint8 CUDA tensor."""
     torch = _torch()
+    pp = _dev(planes, "planes", _dt("uint8"), "slice_prefix")
     out = torch.empty((N, K), dtype=torch.uint8, device=planes.device)
-    check(matq_slice(_ptr(planes), N, K, r_keep, r, _ptr(out), _stream_ptr(stream)), "matq_slice")
+    check(matq_slice(pp, N, K, r_keep, r, _ptr(out), _stream_ptr(stream)), "matq_slice")
     return out
 
 
 def slice_copy(planes, N: int, K: int, r_keep: int, r: int, stream=None):
     """Deployment mode A: a new plane buffer holding only the width-r prefix."""
     torch = _torch()
+    pp = _dev(planes, "planes", _dt("uint8"), "slice_copy")
     nbytes = matq_packed_bytes(N, K, r)
     out = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=planes.device)
-    check(matq_slice_copy(_ptr(planes), N, K, r_keep, r, _ptr(out), out.numel(), _stream_ptr(stream)),
+    check(matq_slice_copy(pp, N, K, r_keep, r, _ptr(out), out.numel(), _stream_ptr(stream)),
           "matq_slice_copy")
     return out[:nbytes]
 
@@ -152,7 +173,8 @@ def workspace(M: int, K: int, N: int, group: int, device="cuda"):
 def workspace_status(ws) -> int:
     """Device status word of a workspace (0 = every call so far completed normally)."""
     out = _c_int(0)
-    check(matq_workspace_status(_ptr(ws), ctypes.byref(out)), "matq_workspace_status")
+    check(matq_workspace_status(_dev(ws, "workspace", _dt("uint8"), "workspace_status"), ctypes.byref(out)),
+          "matq_workspace_status")
     return int(out.value)
 
 
@@ -168,8 +190,12 @@ def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=
         y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, cols), dtype=dt, device=x.device)
     if workspace is None:
         workspace = torch.zeros(max(workspace_bytes(M, K, N, group), 256), dtype=torch.uint8, device=x.device)
-    check(matq_linear(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
-                      _ptr(y), y_mode, _ptr(workspace), workspace.numel(), _stream_ptr(stream)), "matq_linear")
+    w = "linear"
+    ydt = _dt("bfloat16") if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else _dt("float32")
+    check(matq_linear(_dev(x, "x", _dt("bfloat16"), w), M, K, _dev(planes, "planes", _dt("uint8"), w), r_keep,
+                      _dev(scales, "scales", _dt("float16", "int16"), w), _dev(zeros, "zeros", _dt("uint8"), w),
+                      N, r, group, _dev(y, "y", ydt, w), y_mode, _dev(workspace, "workspace", _dt("uint8"), w),
+                      workspace.numel(), _stream_ptr(stream)), "matq_linear")
     return y
 
 
@@ -184,9 +210,13 @@ def linear_noalloc(x, planes, r_keep: int, scales, zeros, N: int, r: int, group:
         dt = torch.bfloat16 if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else torch.float32
         cols = N // 2 if y_mode == MATQ_OUT_SILU_GATED else N
         y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, cols), dtype=dt, device=x.device)
-    sp = _ptr(status) if status is not None else None
-    check(matq_linear_noalloc(_ptr(x), M, K, _ptr(planes), r_keep, _ptr(scales), _ptr(zeros), N, r, group,
-                              _ptr(y), y_mode, sp, _stream_ptr(stream)), "matq_linear_noalloc")
+    w = "linear_noalloc"
+    sp = _dev(status, "status", _dt("int32"), w) if status is not None else None
+    ydt = _dt("bfloat16") if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else _dt("float32")
+    check(matq_linear_noalloc(_dev(x, "x", _dt("bfloat16"), w), M, K, _dev(planes, "planes", _dt("uint8"), w),
+                              r_keep, _dev(scales, "scales", _dt("float16", "int16"), w),
+                              _dev(zeros, "zeros", _dt("uint8"), w), N, r, group, _dev(y, "y", ydt, w), y_mode, sp,
+                              _stream_ptr(stream)), "matq_linear_noalloc")
     return y
 
 
@@ -195,7 +225,8 @@ def rmsnorm(h, eps: float = 1e-5, out=None, stream=None):
     M, D = h.shape
     if out is None:
         out = torch.empty((M, D), dtype=torch.bfloat16, device=h.device)
-    check(matq_rmsnorm(_ptr(h), M, D, eps, _ptr(out), _stream_ptr(stream)), "matq_rmsnorm")
+    check(matq_rmsnorm(_dev(h, "h", _dt("float32"), "rmsnorm"), M, D, eps,
+                       _dev(out, "out", _dt("bfloat16"), "rmsnorm"), _stream_ptr(stream)), "matq_rmsnorm")
     return out
 
 
@@ -204,7 +235,11 @@ def silu_mul(gate, up, out=None, stream=None):
     M, F = gate.shape
     if out is None:
         out = torch.empty((M, F), dtype=torch.bfloat16, device=gate.device)
-    check(matq_silu_mul(_ptr(gate), _ptr(up), M, F, _ptr(out), _stream_ptr(stream)), "matq_silu_mul")
+    if tuple(up.shape) != (M, F):
+        raise ValueError("silu_mul: gate and up must have the same shape")
+    b = _dt("bfloat16")
+    check(matq_silu_mul(_dev(gate, "gate", b, "silu_mul"), _dev(up, "up", b, "silu_mul"), M, F,
+                        _dev(out, "out", b, "silu_mul"), _stream_ptr(stream)), "matq_silu_mul")
     return out
 
 
@@ -215,5 +250,9 @@ def silu_mul_gu(gu, out=None, stream=None):
     F = F2 // 2
     if out is None:
         out = torch.empty((M, F), dtype=torch.bfloat16, device=gu.device)
-    check(matq_silu_mul_gu(_ptr(gu), M, F, _ptr(out), _stream_ptr(stream)), "matq_silu_mul_gu")
+    if F2 % 2:
+        raise ValueError("silu_mul_gu: gu must have an even number of columns")
+    b = _dt("bfloat16")
+    check(matq_silu_mul_gu(_dev(gu, "gu", b, "silu_mul_gu"), M, F, _dev(out, "out", b, "silu_mul_gu"),
+                           _stream_ptr(stream)), "matq_silu_mul_gu")
     return out

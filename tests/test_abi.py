@@ -123,3 +123,21 @@ def test_glue_rejects(M):
     assert M.matq_silu_mul_gu(FAKE, 1, 0, FAKE, None) == M.MATQ_EINVAL_SHAPE
     assert M.matq_silu_mul_gu(None, 1, 16, FAKE, None) == M.MATQ_ENULL
     assert M.matq_silu_mul_gu(FAKE + 2, 1, 16, FAKE, None) == M.MATQ_EALIGN
+
+
+def test_binding_rejects_host_and_strided_tensors(M):
+    """The tensor helpers refuse what the C ABI cannot detect itself (before any CUDA call):
+    host memory, which a kernel would fault on, and wrong element types."""
+    import torch
+    x = torch.zeros((1, 256), dtype=torch.bfloat16)
+    planes = torch.zeros(4096, dtype=torch.uint8)
+    s = torch.zeros((16, 2), dtype=torch.int16)
+    z = torch.zeros((16, 2), dtype=torch.uint8)
+    y = torch.zeros((1, 16), dtype=torch.bfloat16)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        M.linear(x, planes, 8, s, z, 16, 4, 128, y=y, workspace=ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        M.pack(torch.zeros((16, 256), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        M.silu_mul_gu(torch.zeros((1, 32), dtype=torch.bfloat16), out=torch.zeros((1, 16), dtype=torch.bfloat16))
