@@ -45,20 +45,27 @@ pack_kernel(const uint8_t* __restrict__ codes, PlaneGeom g, int nplanes, uint8_t
 
   const int gid = lane >> 2, tg = lane & 3;
   // 2-bit planes: 8 words per lane; 1-bit planes: 4 words per lane.
+  // The fields f0, f0 + 4, f0 + 8, f0 + 12 of a block (f0 = 0..3) lie 8 bits apart in every
+  // plane word (bits 2f of 2-bit words, 4*(f >> 1) + 2a + (f & 1) of 1-bit words), and their
+  // codes are bytes k0, k0 + 16, k0 + 1, k0 + 17 of one row (k0 = 32w + 2tg + 8*(f0 >> 1),
+  // row gid + 8*(f0 & 1)).  One byte permute gathers the four codes into X; each plane then
+  // takes a shift, a mask and an or for four weights at once.
   uint32_t w0[8] = {0}, w3[8] = {0}, w4[8] = {0}, w1[4] = {0}, w2[4] = {0};
 #pragma unroll
   for (int w = 0; w < 8; ++w) {
 #pragma unroll
-    for (int f = 0; f < 16; ++f) {
-      int row, k;
-      field_coords(gid, tg, w, f, row, k);
-      const uint32_t q = tile[row * kPitch + k];
-      w0[w] |= ((q >> 6) & 3u) << (2 * f);
-      w3[w] |= ((q >> 2) & 3u) << (2 * f);
-      w4[w] |= (q & 3u) << (2 * f);
-      const int pos = onebit_pos(w & 1, f);
-      w1[w >> 1] |= ((q >> 5) & 1u) << pos;
-      w2[w >> 1] |= ((q >> 4) & 1u) << pos;
+    for (int f0 = 0; f0 < 4; ++f0) {
+      const uint8_t* rp = tile + (gid + 8 * (f0 & 1)) * kPitch + 32 * w + 2 * tg + 8 * (f0 >> 1);
+      const uint32_t p0 = *reinterpret_cast<const uint16_t*>(rp);
+      const uint32_t p1 = *reinterpret_cast<const uint16_t*>(rp + 16);
+      const uint32_t X = __byte_perm(p0, p1, 0x5140);  // bytes: k0, k0 + 16, k0 + 1, k0 + 17
+      const int s2 = 2 * f0;
+      w0[w] |= ((X >> 6) & 0x03030303u) << s2;
+      w3[w] |= ((X >> 2) & 0x03030303u) << s2;
+      w4[w] |= (X & 0x03030303u) << s2;
+      const int s1 = 4 * (f0 >> 1) + 2 * (w & 1) + (f0 & 1);
+      w1[w >> 1] |= ((X >> 5) & 0x01010101u) << s1;
+      w2[w >> 1] |= ((X >> 4) & 0x01010101u) << s1;
     }
   }
   const size_t t = (size_t)rt * g.KC + kc;
