@@ -7,8 +7,6 @@ M in {1, 4, 16}, one FFN forward through the sliced linears:
            row-interleaved [gate; up] pack, MATQ_OUT_SILU_GATED: the gated product is formed
            in the epilogue from the fp32 results)
     y    = a . W_down,r^T           [M, 4096]
-(on the prefill workload the gate+up call writes both halves, [M, 28672], and matq_silu_mul_gu
-forms the product: there the epilogue arithmetic would compete with the dequantising warps)
 with group-128 parent codes of N(0, 0.02) weights (synthetic, seeded) and N(0, 1) bf16
 activations.  ``value`` = algorithmic bytes of the sliced linears (planes of width r,
 fp16 scales, uint8 zeros, x, y) over the device time of the step -> GB/s.
@@ -90,8 +88,8 @@ FFN_CALLS = (("gate_up", (2 * D_FF, D_MODEL)), ("down", (D_MODEL, D_FF)))
 
 
 def gated_epilogue(spec):
-    """The gated product is fused into the gate+up call on the decode workload only."""
-    return spec["unit"] == "GB/s"
+    """The gated product is fused into the gate+up call (both workloads)."""
+    return True
 
 
 def out_cols(spec, name):
@@ -405,9 +403,9 @@ def run_ours(args):
                            timing="CUDA graph replay, CUDA events"),
             "roofline": rl,
             "e2e": e2e,
-            # per FFN: gated gate+up and down, one kernel each on the decode path; on the prefill
-            # path activation conversion + GEMM each, and the gated product
-            "gpu_launches": args.steps * len(calls) * (len(FFN_CALLS) if gated else 2 * len(FFN_CALLS) + 1),
+            # per FFN: gated gate+up and down, one kernel each on the decode path, activation
+            # conversion + GEMM each on the prefill path
+            "gpu_launches": args.steps * len(calls) * len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2),
             "clocks": clk.summary(),
             "peaks_source": peaks.get("_source"),
         }
@@ -589,10 +587,9 @@ def run_pack_case(args):
 
 
 def run_case(args):
-    """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128;
-    gated-product epilogue for --case decode, both halves written for --case prefill, as in
-    the workloads) at width r and batch m, rotating through device copies of the pack (> L2);
-    used for ncu captures.
+    """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128,
+    gated-product epilogue, as in the workloads) at width r and batch m, rotating through
+    device copies of the pack (> L2); used for ncu captures.
     `--case pack` times the one-time pack instead."""
     if args.case == "pack":
         return run_pack_case(args)
@@ -608,7 +605,7 @@ def run_case(args):
     xb, _ = synth.activations(args.m, D_MODEL, seed=0, outlier_frac=0.01 if args.case == "prefill" else 0.0)
     dx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
     ws = matq.workspace(args.m, D_MODEL, N, GROUP)
-    gated = args.case == "decode"
+    gated = True
     y = torch.empty((args.m, N // 2 if gated else N), dtype=torch.bfloat16, device="cuda")
     mode = matq.MATQ_OUT_SILU_GATED if gated else matq.MATQ_OUT_BF16
     for i in range(args.calls):

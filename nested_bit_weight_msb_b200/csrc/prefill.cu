@@ -399,15 +399,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
         float v[32];
         tmem_ld32(taddr + c * 32, v);
         if (P.y_mode == 3) {
-          // gated mode: even rows (gate) take the odd row below (up) from the next lane and
-          // write silu(gate) * up at column n / 2 of y [M, N/2]
+          // gated mode: lanes 2i (gate row) and 2i + 1 (up row) share output column n / 2 of
+          // y [M, N/2]; the even lane forms tokens 0..15 of the chunk, the odd lane 16..31,
+          // each taking the value it lacks from its partner
+          const bool even = (lane & 1) == 0;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float u = __shfl_down_sync(0xffffffffu, v[k], 1);
-            const int tok = m0 + c * 32 + k;
-            if ((lane & 1) == 0 && n < P.N && tok < P.M)
+          for (int k = 0; k < 16; ++k) {
+            const float other = __shfl_xor_sync(0xffffffffu, even ? v[k + 16] : v[k], 1);
+            const float g = even ? v[k] : other;
+            const float u = even ? other : v[k + 16];
+            const int tok = m0 + c * 32 + k + (even ? 0 : 16);
+            if (n < P.N && tok < P.M)
               reinterpret_cast<__nv_bfloat16*>(P.y)[(size_t)tok * (P.N >> 1) + (n >> 1)] =
-                  __float2bfloat16_rn(__fdividef(v[k], 1.0f + __expf(-v[k])) * u);
+                  __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
           }
         } else if (n < P.N) {
 #pragma unroll
