@@ -439,8 +439,8 @@ _KERNEL_SOURCES = {
 NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
     "decode": {"sha256": "0532170b3041f920007ae78a117291f110bc4db70afbe0a4056be508aefd1756", "launch": "gate_up gated 28672x4096 r=2 M=1",
                "bytes": 32_189_952 + 0},
-    "prefill": {"sha256": "e65082c36fd9bc05759950ee33e9ec7141f7a1b6b9df61b7c7cceafd9d884e25", "launch": "gate_up 28672x4096 r=4 M=2048",
-                "bytes": 78_459_904 + 79_054_848},
+    "prefill": {"sha256": "db3339a9714ea591b690c3e5b188aba3558a03759e92efc1d78c9ba8c6cbd491", "launch": "gate_up gated 28672x4096 r=4 M=2048",
+                "bytes": 78_311_168 + 31_010_048},
 }
 
 
