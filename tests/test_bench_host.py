@@ -60,3 +60,17 @@ def test_both_arms_report_the_same_workload_config():
     assert "gated" in c["shapes"]
     assert "gated" in bench.workload_config(type("A", (), dict(workload="ffn8b_prefill"))(),
                                             bench.workload_spec("ffn8b_prefill"), 1)["shapes"]
+
+
+def test_copy_groups_cover_every_call_once_in_order():
+    # decode-sized inputs (M in {1, 4, 16} rows of 4096 bf16) at five widths: one run per step
+    dec = [m * 4096 * 2 for m in (1, 4, 16)] * 5
+    assert bench.copy_groups(dec) == [list(range(15))]
+    # prefill-sized inputs (M = 2048): one run per call
+    assert bench.copy_groups([2048 * 4096 * 2] * 3) == [[0], [1], [2]]
+    # a run closes at the threshold; the remainder forms the last run
+    assert bench.copy_groups([3, 1, 2, 2, 1], min_bytes=4) == [[0, 1], [2, 3], [4]]
+    assert bench.copy_groups([], min_bytes=4) == []
+    for sizes in ([5, 1, 1, 1, 9, 2], [1] * 7, [10]):
+        flat = [i for g in bench.copy_groups(sizes, min_bytes=4) for i in g]
+        assert flat == list(range(len(sizes)))
