@@ -62,11 +62,22 @@ def quantize_minmax(w, group):
     return q.reshape(N, K).astype(np.uint8), s, z.astype(np.uint8)
 
 
+def _float_w(N, K, seed, layer, proj, std):
+    rng = _rng(seed, layer, PROJ.get(proj, proj), KIND_WEIGHT)
+    return (np.float32(std) * rng.standard_normal((N, K), dtype=np.float32)).astype(np.float32)
+
+
 def parent_weights(N, K, group, seed=0, layer=0, proj="gate", std=0.02):
     """Seeded parent codes [N, K] u8, fp16 scales [N, K/group], u8 zeros [N, K/group]."""
-    rng = _rng(seed, layer, PROJ.get(proj, proj), KIND_WEIGHT)
-    w = (np.float32(std) * rng.standard_normal((N, K), dtype=np.float32)).astype(np.float32)
-    return quantize_minmax(w, group)
+    return quantize_minmax(_float_w(N, K, seed, layer, proj, std), group)
+
+
+def float_weights(N, K, group, seed=0, layer=0, proj="gate", std=0.02):
+    """The fp32 weights [N, K] behind parent_weights (same arguments, same weights) with their
+    per-group MinMax fp16 scales and u8 zero points: the inputs of a parent-code choice."""
+    w = _float_w(N, K, seed, layer, proj, std)
+    _, s, z = quantize_minmax(w, group)
+    return w, s, z
 
 
 def activations(M, K, seed=0, layer=0, proj="gate", outlier_frac=0.0, outlier_mult=20.0):

@@ -6,4 +6,5 @@ baseline / reference legs.  It shares no code with the CUDA library.
 from .matq_oracle import *  # noqa: F401,F403
 from .matq_oracle import (C_BITS, WIDTHS, MODES, prefix, delta, reconstruct, dequant,  # noqa: F401
                           linear, linear_loops, linear_group_sums, bits_read_per_weight,
-                          rmsnorm, silu, gated_product, ffn_block, mixnmatch_effective_bits)
+                          rmsnorm, silu, gated_product, ffn_block, mixnmatch_effective_bits,
+                          choose_codes)

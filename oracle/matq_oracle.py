@@ -39,6 +39,12 @@ Pages are cited by title and section.
   and the zero point applied to the per-group activation sums (App. A.1: delta
   can be absorbed into the zero point).  Exact algebra, checked against
   ``linear``.
+* ``choose_codes`` -- the parent code of each weight chosen for several widths
+  at once: every candidate code is dequantised at each target width with the
+  shared scale and zero point, and the lambda-weighted sum of squared errors
+  decides (MatGPTQ §3.2 item 2, App. A.2 Algorithm 2, brute force over all 2^c
+  candidates, fp32 as the page keeps the candidate errors).  lambda is an
+  input: the pages do not print the values they used.
 * ``rmsnorm``, ``silu``, ``ffn_block`` -- the glue of the Mix'n'Match stack
   ("Matryoshka Quantization | Summary", §4.3 Layerwise Mix'n'Match; MatGPTQ
   §5.4).  The pages give no block formula; the reading taken is a Llama-style
@@ -276,3 +282,55 @@ def mixnmatch_effective_bits(widths, sizes=None):
         return float(widths.mean())
     sizes = np.asarray(sizes, dtype=np.float64)
     return float((widths * sizes).sum() / sizes.sum())
+
+
+def choose_codes(w, scale, zero, group, widths=(3, 4, 8), lambdas=None, mode="true_prefix"):
+    """Parent codes chosen for several widths at once ("MatGPTQ: Efficient and Accurate
+    Inference over Nested Quantized Models", §3.2 item 2 and App. A.2, the brute-force
+    quant_MatGPTQ step of Algorithm 2).
+
+    Every weight w[n, k] tries all 2^c candidate codes q.  Each candidate is dequantised at
+    every target width r with the weight's shared group scale s and zero point z,
+    w_hat_r(q) = s * (reconstruct(q, r, mode) - z), and scored with
+    lambda_r * (w - w_hat_r(q))^2, summed over the widths in the order given.  The code with
+    the smallest total is kept; on a tie the smallest code (argmin's first occurrence).
+
+    Arithmetic: fp32 with every operation rounded on its own, the precision the page gives
+    for the candidate errors (App. A.2, runtime and memory: the 2^c x rows matrix is held in
+    FP32).  w_hat_r is exact in fp32 (an 11-bit scale times a half-integer below 256), so the
+    roundings are those of e = w - w_hat_r, e * e, lambda_r * (e * e) and the running sum.
+
+    widths: strictly ascending widths from WIDTHS.  lambdas: one finite non-negative weight
+    per width (default: equal weights summing to one, the normalised lambda of §3.2 item 3).
+    Returns uint8 codes [N, K].
+    """
+    widths = tuple(int(r) for r in widths)
+    if not widths or any(r not in WIDTHS for r in widths) or any(a >= b for a, b in zip(widths, widths[1:])):
+        raise ValueError("widths must be a strictly ascending subset of (2, 3, 4, 6, 8)")
+    if lambdas is None:
+        lambdas = [1.0 / len(widths)] * len(widths)
+    lam = np.asarray(lambdas, dtype=np.float32)
+    if lam.shape != (len(widths),) or not np.all(np.isfinite(lam)) or np.any(lam < 0):
+        raise ValueError("one finite, non-negative lambda per width")
+    w32 = np.asarray(w, dtype=np.float32)
+    if w32.ndim != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w32.shape
+    s32 = np.repeat(np.asarray(scale, dtype=np.float16).astype(np.float32), group, axis=1)
+    z32 = np.repeat(np.asarray(zero, dtype=np.uint8).astype(np.float32), group, axis=1)
+    if s32.shape != (N, K) or z32.shape != (N, K):
+        raise ValueError("per-group metadata has the wrong shape")
+    cand = np.arange(1 << C_BITS, dtype=np.uint8)
+    qhat = {r: reconstruct(cand, r, mode).astype(np.float32)[:, None, None] for r in widths}
+    out = np.empty((N, K), dtype=np.uint8)
+    rows = max(1, (1 << 24) // ((1 << C_BITS) * max(K, 1)))  # bounds the candidate matrix
+    for n0 in range(0, N, rows):
+        sl = slice(n0, min(N, n0 + rows))
+        wv, sv, zv = w32[sl][None], s32[sl][None], z32[sl][None]
+        total = None
+        for r, lr in zip(widths, lam):
+            e = wv - sv * (qhat[r] - zv)
+            t = lr * (e * e)
+            total = t if total is None else total + t
+        out[sl] = np.argmin(total, axis=0)
+    return out

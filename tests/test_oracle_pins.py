@@ -320,3 +320,113 @@ def test_bf16_rounding_matches_torch():
     xb, xv = synth.activations(4, 1000, outlier_frac=0.01)
     big = np.abs(xv).max(axis=0)
     assert (big > 10).sum() >= 5
+
+
+# --------------------------------------------------------------------------
+# Parent-code choice for several widths (MatGPTQ §3.2 item 2, App. A.2)
+# --------------------------------------------------------------------------
+
+def _one_weight(mode, s, z, widths, lams, w, group=64):
+    wm = np.zeros((1, group), dtype=np.float32)
+    wm[0, 0] = np.float32(w)
+    return int(O.choose_codes(wm, np.array([[s]], np.float16), np.array([[z]], np.uint8), group,
+                              widths, lams, mode)[0, 0])
+
+
+def test_code_choice_hand_examples(golden):
+    rows = golden("matgptq_code_choice.txt")
+    assert len(rows) == 11
+    for mode, s, z, widths, lams, w, want in rows:
+        widths = tuple(int(v) for v in widths.split(","))
+        lams = [float(v) for v in lams.split(",")]
+        assert _one_weight(mode, float(s), int(z), widths, lams, float(w)) == int(want), (mode, widths, lams, w)
+
+
+def _choice_problem(N=48, K=256, group=64, seed=5, spread=1.0):
+    w, s, z = synth.float_weights(N, K, group, seed=seed)
+    w = (w * np.float32(spread)).astype(np.float32)
+    u = w.astype(np.float64) / np.repeat(s.astype(np.float64), group, axis=1) + np.repeat(z, group, axis=1)
+    return w, s, z, u
+
+
+@pytest.mark.parametrize("widths", [(8,), (2, 8), (3, 4, 8), (2, 3, 4, 6, 8), (4, 6, 8)])
+def test_centred_choice_is_round_to_nearest(widths):
+    # With the centred reconstruction the boundary between two cells of any width lies half
+    # way between two 8-bit codes, so the nearest 8-bit code sits in the nearest cell of every
+    # width and minimises every term at once: the choice is round-to-nearest whenever the
+    # 8-bit term carries weight (ties at half-way excluded).  spread > 1 pushes weights past
+    # the grid so the clamps at 0 and 255 are met too.
+    rng = np.random.default_rng(len(widths))
+    for spread in (1.0, 1.6):
+        w, s, z, u = _choice_problem(spread=spread, seed=int(10 * spread))
+        lams = rng.uniform(0.1, 2.0, len(widths)).astype(np.float32)
+        got = O.choose_codes(w, s, z, 64, widths, lams, "true_prefix")
+        want = np.clip(np.floor(u + 0.5), 0, 255)
+        keep = np.abs(u - np.floor(u) - 0.5) > 1e-3
+        assert keep.mean() > 0.99
+        assert np.array_equal(got[keep], want[keep].astype(np.uint8))
+        if spread > 1:
+            assert (want == 0).any() and (want == 255).any()
+
+
+@pytest.mark.parametrize("r", [2, 3, 4, 6])
+@pytest.mark.parametrize("mode", ["true_prefix", "truncate"])
+def test_single_width_choice_is_smallest_code_of_nearest_cell(r, mode):
+    # one width below 8: every code of a cell scores the same, so the smallest code of the
+    # cell whose reconstruction is nearest wins
+    w, s, z, u = _choice_problem(seed=7, spread=1.3)
+    got = O.choose_codes(w, s, z, 64, (r,), None, mode)
+    step = 1 << (8 - r)
+    off = (step - 1) / 2 if mode == "true_prefix" else 0.0
+    v = (u - off) / step
+    p = np.clip(np.floor(v + 0.5), 0, (1 << r) - 1)
+    keep = np.abs(v - np.floor(v) - 0.5) > 1e-4
+    assert np.array_equal(got[keep], (p[keep] * step).astype(np.uint8))
+    assert np.all(got % step == 0)
+
+
+@pytest.mark.parametrize("r", [2, 3, 4, 6])
+def test_truncated_two_width_choice_by_cells(r):
+    # Raw truncation, widths {r, 8}: a different algorithm in fp64 -- per cell of width r the
+    # best code is the nearest code clamped into the cell, the cell's cost is
+    # lam_r*(u - edge)^2 + lam_8*(u - code)^2, and the cheapest cell wins.  Near-ties between
+    # cells and half-way codes are excluded.
+    w, s, z, u = _choice_problem(N=32, seed=9, spread=1.2)
+    lam = np.array([0.7, 1.3], dtype=np.float32)
+    got = O.choose_codes(w, s, z, 64, (r, 8), lam, "truncate")
+    step = 1 << (8 - r)
+    edges = np.arange(1 << r, dtype=np.float64) * step
+    uu = u[..., None]
+    code = np.clip(np.floor(uu + 0.5), edges, edges + step - 1)
+    cost = float(lam[0]) * (uu - edges) ** 2 + float(lam[1]) * (uu - code) ** 2
+    order = np.sort(cost, axis=-1)
+    best = np.argmin(cost, axis=-1)
+    want = np.take_along_axis(code, best[..., None], axis=-1)[..., 0]
+    keep = (order[..., 1] - order[..., 0] > 1e-6 * (1 + order[..., 0])) & (np.abs(u - np.floor(u) - 0.5) > 1e-4)
+    assert keep.mean() > 0.95
+    assert np.array_equal(got[keep], want[keep].astype(np.uint8))
+    # the trade-off is real: some weights leave the nearest code
+    assert (got != np.clip(np.floor(u + 0.5), 0, 255)).mean() > 0.05
+
+
+def test_code_choice_lambda_properties():
+    w, s, z, _ = _choice_problem(N=16, seed=11)
+    base = O.choose_codes(w, s, z, 64, (2, 4, 8), [0.25, 0.5, 1.0], "truncate")
+    # a power-of-two scale of every lambda scales every fp32 total exactly
+    assert np.array_equal(base, O.choose_codes(w, s, z, 64, (2, 4, 8), [1.0, 2.0, 4.0], "truncate"))
+    # zero weights drop their widths (0 + 0 + t == t exactly)
+    only8 = O.choose_codes(w, s, z, 64, (8,), [1.0], "truncate")
+    assert np.array_equal(only8, O.choose_codes(w, s, z, 64, (2, 4, 8), [0, 0, 1], "truncate"))
+    only2 = O.choose_codes(w, s, z, 64, (2,), [1.0], "truncate")
+    assert np.array_equal(only2, O.choose_codes(w, s, z, 64, (2, 4, 8), [1, 0, 0], "truncate"))
+    assert not np.array_equal(only2, only8)
+    # every lambda zero: all totals tie and the smallest code wins
+    assert not O.choose_codes(w, s, z, 64, (3, 8), [0, 0], "truncate").any()
+
+
+def test_code_choice_is_validated():
+    w, s, z, _ = _choice_problem(N=2, K=64)
+    for widths, lams in (((8, 4), None), ((4, 4), None), ((5,), None), ((), None), ((4, 8), [1, -1]),
+                         ((4, 8), [1]), ((4, 8), [1, float("nan")])):
+        with pytest.raises(ValueError):
+            O.choose_codes(w, s, z, 64, widths, lams)
