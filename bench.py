@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
     ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "prefill", "pack"], default=None,
+    ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
     ap.add_argument("--m", type=int, default=1)
@@ -657,11 +657,56 @@ def run_pack_case(args):
     return 0
 
 
+def run_choose_case(args):
+    """The parent-code choice for several widths (matq_choose_codes) on every 8B and 9B FFN
+    matrix: widths {3, 4, 8} with equal lambdas (the pages' width set), centred and truncated
+    reconstruction, timed with CUDA events over 10 back-to-back calls each (the fp32 weights,
+    > 200 MB a matrix, exceed L2).  Reports weights per second and GB/s of the call's bytes
+    (4 B of w read + 1 B of code written per weight, 3 B of scale and zero point per group)
+    against the measured copy peak; the search itself is fp32 ALU work."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq, synth
+    torch.cuda.set_device(0)
+    peaks = load_peaks()
+    out = {}
+    for name, (N, K, g) in (("8b gate/up", (14336, 4096, 128)), ("8b down", (4096, 14336, 128)),
+                            ("9b gate/up", (14336, 3584, 64)), ("9b down", (3584, 14336, 64))):
+        w, s, z = synth.float_weights(N, K, g, seed=0)
+        dw = torch.from_numpy(w).cuda()
+        ds = torch.from_numpy(s.view(np.int16)).cuda()
+        dz = torch.from_numpy(z).cuda()
+        codes = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+        for mode, mname in ((matq.MATQ_SLICE_TRUE_PREFIX, "true_prefix"), (matq.MATQ_SLICE_TRUNCATE, "truncate")):
+            def call():
+                matq.choose_codes(dw, ds, dz, g, (3, 4, 8), None, mode, out=codes)
+            for _ in range(3):
+                call()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            n = 10
+            e0.record()
+            for _ in range(n):
+                call()
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) / n * 1e3
+            nbytes = N * K * 5 + N * (K // g) * 3
+            out[f"{name} {mname}"] = {"us": round(us, 1), "Gweights/s": round(N * K / us / 1e3, 1),
+                                      "GB/s": round(nbytes / us / 1e3, 1),
+                                      "frac_of_copy_peak": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 3)}
+    print(json.dumps({"case": "choose", "widths": [3, 4, 8], "lambdas": "equal", "results": out,
+                      "peak_hbm_gbs": peaks["hbm_gbs"], "peaks_source": peaks["_source"]}))
+    return 0
+
+
 def run_case(args):
     """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128,
     gated-product epilogue, as in the workloads) at width r and batch m, rotating through
     device copies of the pack (> L2); used for ncu captures.
     `--case pack` times the one-time pack instead."""
+    if args.case == "choose":
+        return run_choose_case(args)
     if args.case == "pack":
         return run_pack_case(args)
     import torch

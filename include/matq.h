@@ -27,7 +27,8 @@
  *   - Every call returns an int status: MATQ_OK (0) or a negative MATQ_E* code.  Argument
  *     errors are caught on the host before any launch and leave every buffer untouched.
  *     A launch failure returns MATQ_ECUDA; matq_last_cuda_error() gives the cudaError_t.
- *   - Shapes: N >= 1; K a positive multiple of 256; M >= 1.  group in {64, 128}.
+ *   - Shapes: N >= 1; K a positive multiple of 256 (matq_choose_codes: of group); M >= 1.
+ *     group in {64, 128}.
  *   - Alignment: every device pointer must be 16-byte aligned.
  *   - Thread safety: calls on different streams may run concurrently; the only state is a
  *     thread-local "last CUDA error".
@@ -82,6 +83,7 @@ extern "C" {
 #define MATQ_EDTYPE        -9   /* unknown output mode                                      */
 #define MATQ_EDEVICE      -10   /* current device is not sm_100 (B200 class)               */
 #define MATQ_ESCRATCH     -11   /* sizes exceed matq_linear_noalloc's fixed scratch        */
+#define MATQ_EINVAL_ARG   -12   /* a lambda < 0 or not finite, or an unknown slicing mode  */
 
 /* ---- output modes of matq_linear ----------------------------------------------------- */
 #define MATQ_OUT_BF16       0   /* y [M, N] bf16 = x . W_hat^T                             */
@@ -222,6 +224,42 @@ int matq_linear_noalloc(const void* x, int M, int K,
                         int r, int group,
                         void* y, int y_mode,
                         int* status_out, void* stream);
+
+/* ---- parent-code choice for several widths -------------------------------------------- */
+
+/* Reconstruction rules a code choice can score with ("MatGPTQ" App. A.1). */
+#define MATQ_SLICE_TRUE_PREFIX 0   /* q_hat = p * 2^(8-r) + (2^(8-r) - 1) / 2 (centred)     */
+#define MATQ_SLICE_TRUNCATE    1   /* q_hat = p * 2^(8-r) (raw MSB truncation)               */
+
+/* matq_choose_codes -- the parent code of every weight, chosen for several widths at once
+ * ("MatGPTQ: Efficient and Accurate Inference over Nested Quantized Models", §3.2 item 2 and
+ * App. A.2, Algorithm 2: the quant_MatGPTQ step).  Each weight w[n][k] gets the code q in
+ * [0, 255] that minimises
+ *     total(q) = sum_i lambdas[i] * (w - s * (q_hat_{widths[i]}(q) - z))^2
+ * with s, z the weight's group scale and zero point and q_hat the rule of slice_mode.  The
+ * arithmetic is fp32 with every operation rounded on its own (s * (q_hat - z) is exact; then
+ * e = w - that, e * e, lambda * (e * e), and the running sum, terms added in the order of
+ * `widths`), the precision the page gives for its candidate errors; on a tie the smallest
+ * code wins (the first minimum of an argmin over q = 0..255).  Non-finite inputs or s <= 0
+ * follow the same definition (an argmin meeting NaN totals takes the first NaN).
+ * The page runs this per column inside GPTQ, on weights that error feedback has updated;
+ * this call applies it to a whole matrix as given (the Hessian pass that produces those
+ * weights needs calibration data and is not part of libmatq).  With MATQ_SLICE_TRUE_PREFIX
+ * and a positive weight on width 8 the result is round-to-nearest (cell boundaries of every
+ * width fall half way between two codes); raw truncation makes the widths trade off.
+ *   w        fp32 [N, K] row-major (device).
+ *   scales   fp16 [N, K/group], zeros uint8 [N, K/group] (device), as matq_linear takes them.
+ *   group    64 or 128; K a positive multiple of group (K need not be a multiple of 256).
+ *   n_widths 1..5; widths: HOST array, strictly ascending, each in {2, 3, 4, 6, 8}.
+ *   lambdas  HOST array of n_widths finite, non-negative weights (the pages do not print the
+ *            values they used; equal weights summing to one are a neutral choice).
+ *   codes    uint8 [N, K] (device): the chosen parent codes, ready for matq_pack.
+ * Errors: MATQ_EINVAL_GROUP, MATQ_EINVAL_SHAPE, MATQ_ENULL, MATQ_EINVAL_R (widths),
+ * MATQ_EINVAL_ARG (lambdas, slice_mode), MATQ_EALIGN, MATQ_EDEVICE, MATQ_ECUDA. */
+int matq_choose_codes(const float* w, int N, int K,
+                      const uint16_t* scales, const uint8_t* zeros, int group,
+                      int n_widths, const int* widths, const float* lambdas, int slice_mode,
+                      uint8_t* codes, void* stream);
 
 /* ---- glue of the Mix'n'Match FFN stack ------------------------------------------------- */
 

@@ -5,6 +5,7 @@
 #include <stddef.h>
 
 #include <atomic>
+#include <cmath>
 
 #include "../../include/matq.h"
 #include "common.cuh"
@@ -100,6 +101,7 @@ const char* matq_strerror(int status) {
     case MATQ_ESCRATCH:
       return "sizes need more scratch than matq_linear_noalloc's fixed array (MATQ_NOALLOC_SCRATCH_BYTES); "
              "use matq_linear with a caller workspace";
+    case MATQ_EINVAL_ARG: return "invalid argument (a lambda negative or not finite, or an unknown slicing mode)";
     default: return "unknown status";
   }
 }
@@ -222,6 +224,26 @@ int matq_silu_mul_gu(const void* gu, int M, int F, void* a_out, void* stream) {
   int st = check_device();
   if (st) return st;
   return cuda_status(launch_silu_mul_gu(gu, M, F, a_out, (cudaStream_t)stream));
+}
+
+int matq_choose_codes(const float* w, int N, int K, const uint16_t* scales, const uint8_t* zeros, int group,
+                      int n_widths, const int* widths, const float* lambdas, int slice_mode, uint8_t* codes,
+                      void* stream) {
+  if (group != 64 && group != 128) return MATQ_EINVAL_GROUP;
+  if (N < 1 || K < group || K % group != 0 || (long long)N * (long long)K > (1LL << 40)) return MATQ_EINVAL_SHAPE;
+  if (!widths || !lambdas) return MATQ_ENULL;
+  if (n_widths < 1 || n_widths > 5) return MATQ_EINVAL_R;
+  for (int i = 0; i < n_widths; ++i)
+    if (!valid_width(widths[i]) || (i > 0 && widths[i] <= widths[i - 1])) return MATQ_EINVAL_R;
+  for (int i = 0; i < n_widths; ++i)
+    if (!(lambdas[i] >= 0.f) || !std::isfinite(lambdas[i])) return MATQ_EINVAL_ARG;
+  if (slice_mode != MATQ_SLICE_TRUE_PREFIX && slice_mode != MATQ_SLICE_TRUNCATE) return MATQ_EINVAL_ARG;
+  if (!w || !scales || !zeros || !codes) return MATQ_ENULL;
+  if (!aligned16(w) || !aligned16(scales) || !aligned16(zeros) || !aligned16(codes)) return MATQ_EALIGN;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_choose(w, N, K, scales, zeros, group, n_widths, widths, lambdas,
+                                   slice_mode == MATQ_SLICE_TRUNCATE, codes, (cudaStream_t)stream));
 }
 
 int matq_silu_mul(const void* gate, const void* up, int M, int F, void* a_out, void* stream) {

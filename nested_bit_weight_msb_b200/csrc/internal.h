@@ -26,6 +26,9 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
 cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s);
 cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s);
 cudaError_t launch_silu_mul_gu(const void* gu, int M, int F, void* out, cudaStream_t s);
+cudaError_t launch_choose(const float* w, int N, int K, const uint16_t* scales, const uint8_t* zeros, int group,
+                          int n_widths, const int* widths, const float* lambdas, int truncate, uint8_t* codes,
+                          cudaStream_t s);
 
 // Host-side per-device caches (api.cu): the SM count of the current device, and the device
 // index with which a launcher records that a kernel's shared-memory attribute is set.

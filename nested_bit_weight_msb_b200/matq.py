@@ -36,10 +36,13 @@ MATQ_ESIZE = -8
 MATQ_EDTYPE = -9
 MATQ_EDEVICE = -10
 MATQ_ESCRATCH = -11
+MATQ_EINVAL_ARG = -12
 MATQ_OUT_BF16 = 0
 MATQ_OUT_F32 = 1
 MATQ_OUT_F32_ACCUM = 2
 MATQ_OUT_SILU_GATED = 3
+MATQ_SLICE_TRUE_PREFIX = 0
+MATQ_SLICE_TRUNCATE = 1
 
 WIDTHS = (2, 3, 4, 6, 8)
 DECODE_MAX_M = 16
@@ -65,6 +68,8 @@ _SIGNATURES = {
     "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
     "matq_silu_mul": (_c_int, [_c_vp, _c_vp, _c_int, _c_int, _c_vp, _c_vp]),
     "matq_silu_mul_gu": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_vp]),
+    "matq_choose_codes": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_vp, _c_int, _c_int, ctypes.POINTER(_c_int),
+                                   ctypes.POINTER(_c_float), _c_int, _c_vp, _c_vp]),
 }
 
 for _name, (_res, _args) in _SIGNATURES.items():
@@ -255,4 +260,31 @@ def silu_mul_gu(gu, out=None, stream=None):
     b = _dt("bfloat16")
     check(matq_silu_mul_gu(_dev(gu, "gu", b, "silu_mul_gu"), M, F, _dev(out, "out", b, "silu_mul_gu"),
                            _stream_ptr(stream)), "matq_silu_mul_gu")
+    return out
+
+
+def choose_codes(w, scales, zeros, group: int, widths=(3, 4, 8), lambdas=None,
+                 mode: int = MATQ_SLICE_TRUE_PREFIX, out=None, stream=None):
+    """Parent codes [N, K] uint8 chosen for several widths at once (matq_choose_codes).
+
+    w fp32 [N, K], scales fp16 [N, K/group] and zeros uint8 [N, K/group] are CUDA tensors;
+    widths (ascending) and lambdas are host sequences, lambdas defaulting to equal weights
+    that sum to one."""
+    torch = _torch()
+    N, K = w.shape
+    widths = [int(r) for r in widths]
+    if lambdas is None:
+        lambdas = [1.0 / len(widths)] * len(widths)
+    lambdas = [float(v) for v in lambdas]
+    if len(lambdas) != len(widths):
+        raise ValueError("choose_codes: one lambda per width")
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    what = "choose_codes"
+    rw = (_c_int * len(widths))(*widths)
+    lw = (_c_float * len(lambdas))(*lambdas)
+    check(matq_choose_codes(_dev(w, "w", _dt("float32"), what), N, K,
+                            _dev(scales, "scales", _dt("float16", "int16"), what),
+                            _dev(zeros, "zeros", _dt("uint8"), what), group, len(widths), rw, lw, mode,
+                            _dev(out, "out", _dt("uint8"), what), _stream_ptr(stream)), "matq_choose_codes")
     return out

@@ -141,3 +141,40 @@ def test_binding_rejects_host_and_strided_tensors(M):
         M.pack(torch.zeros((16, 256), dtype=torch.uint8))
     with pytest.raises(ValueError, match="CUDA tensor"):
         M.silu_mul_gu(torch.zeros((1, 32), dtype=torch.bfloat16), out=torch.zeros((1, 16), dtype=torch.bfloat16))
+
+
+def test_choose_codes_rejects(M):
+    import ctypes
+
+    def call(N=4, K=128, group=64, widths=(3, 4, 8), lams=(1, 1, 1), mode=0, w=FAKE, s=FAKE, z=FAKE, out=FAKE,
+             n=None):
+        rw = (ctypes.c_int * max(1, len(widths)))(*widths) if widths is not None else None
+        lw = (ctypes.c_float * max(1, len(lams)))(*lams) if lams is not None else None
+        nw = len(widths) if (n is None and widths is not None) else (n or 0)
+        return M.matq_choose_codes(w, N, K, s, z, group, nw, rw, lw, mode, out, None)
+
+    assert call(group=32) == M.MATQ_EINVAL_GROUP
+    assert call(N=0) == M.MATQ_EINVAL_SHAPE
+    assert call(K=96) == M.MATQ_EINVAL_SHAPE
+    assert call(K=32) == M.MATQ_EINVAL_SHAPE
+    assert call(widths=None) == M.MATQ_ENULL
+    assert call(lams=None) == M.MATQ_ENULL
+    assert call(widths=(), lams=(), n=0) == M.MATQ_EINVAL_R
+    assert call(widths=(2, 3, 4, 6, 8, 8), lams=(1,) * 6) == M.MATQ_EINVAL_R
+    assert call(widths=(8, 4), lams=(1, 1)) == M.MATQ_EINVAL_R
+    assert call(widths=(4, 4), lams=(1, 1)) == M.MATQ_EINVAL_R
+    assert call(widths=(5,), lams=(1,)) == M.MATQ_EINVAL_R
+    assert call(lams=(1, -1, 1)) == M.MATQ_EINVAL_ARG
+    assert call(lams=(1, float("nan"), 1)) == M.MATQ_EINVAL_ARG
+    assert call(lams=(1, float("inf"), 1)) == M.MATQ_EINVAL_ARG
+    assert call(mode=2) == M.MATQ_EINVAL_ARG
+    assert call(w=None) == M.MATQ_ENULL
+    assert call(out=None) == M.MATQ_ENULL
+    assert call(w=FAKE + 4) == M.MATQ_EALIGN
+    assert call(out=FAKE + 1) == M.MATQ_EALIGN
+    assert call(z=FAKE + 8) == M.MATQ_EALIGN
+    assert "lambda" in M.matq_strerror(M.MATQ_EINVAL_ARG).decode()
+    import torch
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        M.choose_codes(torch.zeros((4, 128)), torch.zeros((4, 2), dtype=torch.float16),
+                       torch.zeros((4, 2), dtype=torch.uint8), 64)
