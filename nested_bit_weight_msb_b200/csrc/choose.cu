@@ -92,8 +92,10 @@ __device__ __forceinline__ uint8_t choose_cells(float w, float s, float z, const
   // minimum over the cell whose finest levels are lo .. lo + per_cell - 1, partial sum S
   auto cell = [&](int lo, float S) {
     const int hi = lo + per_cell - 1;
+    // the minimum over all levels is at p* or p* + 1 (p* the last level with w_hat <= w), and
+    // the estimate pu is one of the two: the levels next to it (clamped to the cell) hold it
     const int pc = min(max(pu, lo), hi);
-    const int a = max(lo, pc - 2), b = min(hi, pc + 2);
+    const int a = max(lo, pc - 1), b = min(hi, pc + 1);
     auto total = [&](float pf) {
       const float t = term(F, pf);
       return NW >= 2 ? __fadd_rn(S, t) : t;
@@ -129,17 +131,28 @@ __device__ __forceinline__ uint8_t choose_cells(float w, float s, float z, const
     // the cell of the nearest finest level first: it usually holds the answer and prunes the rest
     const int c0 = min(max(pu, 0), nf - 1) >> (rf - rc);
     cell(c0 * per_cell, partial(c0, term(0, (float)(c0 >> (rc - r0)))));
-    float p0f = 0.f;
-    for (int p0 = 0; p0 < (1 << r0); ++p0, p0f += 1.f) {
-      const float t0 = term(0, p0f);
-      if (t0 > best || (t0 == best && p0 * sub * per_cell > best_p)) continue;
+    // Coarsest levels outward from the one holding c0.  t0, a lower bound of every total under
+    // its level, falls up to the level p0* (the last with w_hat <= w) and rises after p0* + 1;
+    // the estimate f0 is within one of p0*, so past f0 + 1 to the right and f0 - 1 to the left
+    // a level that fails its bound is followed only by levels that fail it too.
+    const int n0 = 1 << r0;
+    const int f0 = (int)floorf(fminf(fmaxf(__fdividef(__fsub_rn(w, base[0]), step[0]), -4.f), (float)(n0 + 3)));
+    auto level = [&](int p0, bool right) {      // true: the bound rules the level out
+      const float t0 = term(0, (float)p0);
+      if (t0 > best || (right && t0 == best && p0 * sub * per_cell > best_p)) return true;
       for (int c = p0 * sub; c < (p0 + 1) * sub; ++c) {
         if (c == c0) continue;
         const float S = partial(c, t0);
         if (S > best || (S == best && c * per_cell > best_p)) continue;
         cell(c * per_cell, S);
       }
-    }
+      return false;
+    };
+    const int p0c = c0 >> (rc - r0);
+    for (int p0 = p0c; p0 < n0; ++p0)
+      if (level(p0, true) && p0 >= f0 + 2) break;
+    for (int p0 = p0c - 1; p0 >= 0; --p0)
+      if (level(p0, false) && p0 <= f0 - 1) break;
   }
   return (uint8_t)(best_p << (8 - rf));
 }
