@@ -144,11 +144,15 @@ def test_gated_output_mode_8b_sampled(M, Mt):
         assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-6), f"gated epilogue M={Mt} r={r}: {err.max():.3g}"
 
 
+@pytest.mark.parametrize("alloc", ["fixed", "pyramid"])
 @pytest.mark.parametrize("Mt", [1, 16, 40])
-def test_mixnmatch_stack_teacher_forced(M, Mt):
+def test_mixnmatch_stack_teacher_forced(M, Mt, alloc):
+    """A four-layer stack with one width per layer: a fixed mix, and the Pyramid allocation of
+    4 effective bits over widths {2, 4, 8} (middle layers widest)."""
     import torch
+    from nested_bit_weight_msb_b200 import mixnmatch
     D, F, G, L = 512, 1024, 128, 4
-    widths = [2, 4, 3, 8]
+    widths = [2, 4, 3, 8] if alloc == "fixed" else mixnmatch.allocate_widths(L, 4.0, "pyramid", (2, 4, 8))
     layers = []
     for l in range(L):
         lay = {}
