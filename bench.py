@@ -54,7 +54,7 @@ def parse():
     ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
     ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose"], default=None,
+    ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose", "speedup"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
     ap.add_argument("--m", type=int, default=1)
@@ -700,6 +700,65 @@ def run_choose_case(args):
     return 0
 
 
+def run_speedup_case(args):
+    """The pages' own comparison: the sliced linear layer against torch.matmul (cuBLAS) in bf16
+    on a dense weight of the same shape, at the decode batch sizes.  For each 8B FFN matrix and
+    M in {1, 4, 16}: microseconds per call of torch.matmul(x, W^T) and of matq.linear at every
+    width, both as CUDA graphs of 20 back-to-back calls over rotating weight copies (> L2), and
+    the ratio.  Dense weight values do not change cuBLAS's time, so random bf16 values stand in
+    for the dequantised W."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq, synth
+    torch.cuda.set_device(0)
+    copies, calls = 3, 20
+
+    def graph_us(fn):
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            for i in range(3):
+                fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(calls):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / calls * 1e3
+
+    out = {}
+    for name, (N, K) in (("8b gate/up", (D_FF, D_MODEL)), ("8b down", (D_MODEL, D_FF))):
+        dense = [torch.randn((N, K), dtype=torch.bfloat16, device="cuda") for _ in range(copies)]
+        q, s, z = synth.parent_weights(N, K, GROUP, seed=0)
+        p0 = matq.pack(torch.from_numpy(q).cuda(), 8)
+        packs = [p0] + [p0.clone() for _ in range(copies - 1)]
+        ds = torch.from_numpy(s.view(np.int16)).cuda()
+        dz = torch.from_numpy(z).cuda()
+        for M in (1, 4, 16):
+            xb, _ = synth.activations(M, K, seed=0)
+            x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            ws = matq.workspace(M, K, N, GROUP)
+            t_ref = graph_us(lambda i: torch.matmul(x, dense[i % copies].t(), out=y))
+            row = {"torch.matmul bf16 us": round(t_ref, 2)}
+            for r in WIDTHS:
+                t = graph_us(lambda i: matq.linear(x, packs[i % copies], 8, ds, dz, N, r, GROUP, y=y, workspace=ws))
+                row[f"r={r} us"] = round(t, 2)
+                row[f"r={r} speedup"] = round(t_ref / t, 2)
+            out[f"{name} M={M}"] = row
+        del dense, packs
+        torch.cuda.empty_cache()
+    print(json.dumps({"case": "speedup", "baseline": "torch.matmul bf16 (cuBLAS), dense weight of the same shape",
+                      "results": out}))
+    return 0
+
+
 def run_case(args):
     """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128,
     gated-product epilogue, as in the workloads) at width r and batch m, rotating through
@@ -707,6 +766,8 @@ def run_case(args):
     `--case pack` times the one-time pack instead."""
     if args.case == "choose":
         return run_choose_case(args)
+    if args.case == "speedup":
+        return run_speedup_case(args)
     if args.case == "pack":
         return run_pack_case(args)
     import torch
