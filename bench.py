@@ -657,6 +657,30 @@ def run_pack_case(args):
     return 0
 
 
+def cpu_choose_rate(budget_s=10.0, rows=8):
+    """The oracle's parent-code choice (as it stands: fp32 brute force over all 256 codes) timed
+    on the host cores on a bounded sample: the first `rows` rows of the 8B gate matrix, widths
+    {3, 4, 8}, equal lambdas, centred reconstruction, repeated until `budget_s` is spent."""
+    import oracle as O
+    from nested_bit_weight_msb_b200 import synth
+    w, s, z = synth.float_weights(rows, D_MODEL, GROUP, seed=0)
+    done, n_iter = 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or n_iter == 0:
+        O.choose_codes(w, s, z, GROUP, (3, 4, 8))
+        done += w.size
+        n_iter += 1
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count()
+    try:
+        import threadpoolctl
+        cores = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=cores)
+    except Exception:
+        pass
+    return {"value": done / dt / 1e9, "unit": "Gweights/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {rows} rows of the 8B gate matrix (x {D_MODEL} inputs), {n_iter} pass(es), {dt:.1f} s"}
+
+
 def run_choose_case(args):
     """The parent-code choice for several widths (matq_choose_codes) on every 8B and 9B FFN
     matrix: widths {3, 4, 8} with equal lambdas (the pages' width set), centred and truncated
@@ -695,8 +719,11 @@ def run_choose_case(args):
             out[f"{name} {mname}"] = {"us": round(us, 1), "Gweights/s": round(N * K / us / 1e3, 1),
                                       "GB/s": round(nbytes / us / 1e3, 1),
                                       "frac_of_copy_peak": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 3)}
-    print(json.dumps({"case": "choose", "widths": [3, 4, 8], "lambdas": "equal", "results": out,
-                      "peak_hbm_gbs": peaks["hbm_gbs"], "peaks_source": peaks["_source"]}))
+    line = {"case": "choose", "widths": [3, 4, 8], "lambdas": "equal", "results": out,
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peaks_source": peaks["_source"]}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_choose_rate()
+    print(json.dumps(line))
     return 0
 
 
