@@ -34,50 +34,7 @@ def edge_codes(N, K, seed):
     return q
 
 
-# --- NumPy model of the documented layout ------------------------------------------------
-PLANE_BITS = [2, 1, 1, 2, 2]
-PLANE_LSB = [6, 5, 4, 2, 0]
-PLANES_FOR = {2: 1, 3: 2, 4: 3, 6: 4, 8: 5}
-
-
-def _field_index():
-    gid = np.arange(32) // 4
-    tg = np.arange(32) % 4
-    w = np.arange(8)
-    f = np.arange(16)
-    L, W, F = np.meshgrid(np.arange(32), w, f, indexing="ij")
-    u = F & 7
-    hi = F >> 3
-    j = u >> 2
-    rho = u & 3
-    row = gid[L] + 8 * (rho & 1)
-    k = 32 * W + 16 * j + 2 * tg[L] + 8 * (rho >> 1) + hi
-    return row, k, W, F
-
-
-def layout_model(q, r_keep):
-    N, K = q.shape
-    RT, KC = (N + 15) // 16, K // 256
-    qp = np.zeros((RT * 16, K), dtype=np.int64)
-    qp[:N] = q
-    row, k, W, F = _field_index()            # [32, 8, 16]
-    out = []
-    for p in range(PLANES_FOR[r_keep]):
-        b = PLANE_BITS[p]
-        vals = (qp >> PLANE_LSB[p]) & ((1 << b) - 1)
-        tiles = vals.reshape(RT, 16, KC, 256).transpose(0, 2, 1, 3)   # [RT, KC, 16, 256]
-        v = tiles[:, :, row, k]                                     # [RT, KC, 32, 8, 16]
-        if b == 2:
-            words = (v << (2 * F)).sum(axis=-1).astype(np.uint32)   # [RT, KC, 32, 8]
-            mem = words.reshape(RT, KC, 32, 2, 4).transpose(0, 1, 3, 2, 4)  # [.., half, lane, 4]
-        else:
-            a = W & 1
-            pos = 4 * (F >> 1) + 2 * a + (F & 1)
-            bits = (v << pos).sum(axis=-1)                          # [RT, KC, 32, 8] per block
-            words = (bits[..., 0::2] + bits[..., 1::2]).astype(np.uint32)   # blocks 2v, 2v+1
-            mem = words                                             # [RT, KC, lane, 4]
-        out.append(np.ascontiguousarray(mem).view(np.uint8).reshape(-1))
-    return np.concatenate(out)
+from layout_model import layout_model  # noqa: E402  (NumPy model of the documented layout)
 
 
 # --- tests ----------------------------------------------------------------------------------

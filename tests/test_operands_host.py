@@ -7,10 +7,12 @@ operands.cuh is compiled unchanged next to a host stand-in for common.cuh that g
 bit helpers it uses their documented meaning -- and_or(a, b, c) = (a & b) | c, bitsel(a, b, m)
 = (a & m) | (b & ~m), and the default-mode byte permute of PTX prmt.b32 (each selector nibble
 picks byte n of the 8-byte pool {b:a}, a = bytes 0..3; its top bit replicates that byte's sign).
-The lane words are built here from random codes with the layout of the header text.  Every fp16
-half of every operand register, for every lane, block and width, must equal 1024 + sigma * v
-with v the prefix (r <= 4) or the prefix shifted back (r = 6, 8) of its weight's code, and
-sigma the register's documented power of two.  No GPU needed.
+The lane words are read from the bytes of the NumPy layout model (tests/layout_model.py, written
+from the header text and also the reference for the pack kernel's output) at the lane offsets
+the kernels load them from.  Every fp16 half of every operand register, for every lane, block
+and width, must equal 1024 + sigma * v with v the prefix (r <= 4) or the prefix shifted back
+(r = 6, 8) of its weight's code, and sigma the register's documented power of two.  No GPU
+needed.
 """
 
 import ctypes
@@ -22,6 +24,7 @@ import numpy as np
 import pytest
 
 import oracle as O
+from layout_model import field_coords as _field_coords, layout_model, tile_lane_words
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "nested_bit_weight_msb_b200", "csrc", "operands.cuh")
@@ -117,32 +120,11 @@ def build_host():
     return run
 
 
-# ---- lane words of one 16 x 256 tile, written from the layout text of include/matq.h ----------
+# ---- lane words of one 16 x 256 tile: the bytes of the layout model, read at the lane offsets ----
 
-def _field_coords(gid, tg, w, f):
-    u, hi = f & 7, f >> 3
-    j, rho = u >> 2, u & 3
-    return gid + 8 * (rho & 1), 32 * w + 16 * j + 2 * tg + 8 * (rho >> 1) + hi
-
-
-def _lane_words(codes, gid, tg):
-    """p0[8], p1[4], p2[4], p3[8], p4[8] of lane (gid, tg): 2-bit planes hold field f of block
-    w in bits [2f, 2f+2) of word w; 1-bit planes hold field f of block 2v + a at bit
-    4*(f >> 1) + 2*a + (f & 1) of word v.  Plane bits: {7:6}, {5}, {4}, {3:2}, {1:0}."""
-    p0 = np.zeros(8, np.uint64); p3 = np.zeros(8, np.uint64); p4 = np.zeros(8, np.uint64)
-    p1 = np.zeros(4, np.uint64); p2 = np.zeros(4, np.uint64)
-    for w in range(8):
-        for f in range(16):
-            row, k = _field_coords(gid, tg, w, f)
-            q = int(codes[row, k])
-            p0[w] |= ((q >> 6) & 3) << (2 * f)
-            p3[w] |= ((q >> 2) & 3) << (2 * f)
-            p4[w] |= (q & 3) << (2 * f)
-            v, a = w >> 1, w & 1
-            pos = 4 * (f >> 1) + 2 * a + (f & 1)
-            p1[v] |= ((q >> 5) & 1) << pos
-            p2[v] |= ((q >> 4) & 1) << pos
-    return np.concatenate([p0, p1, p2, p3, p4]).astype(np.uint32)
+def _lane_words_of(codes):
+    tile = layout_model(codes, 8)
+    return {(gid, tg): tile_lane_words(tile, 4 * gid + tg) for gid in range(8) for tg in range(4)}
 
 
 def _sigma(r, rho):
@@ -160,9 +142,10 @@ def test_operands_are_exact_prefix_values(build_host, r):
     codes[0, :16] = [0, 255, 0x55, 0xAA, 1, 2, 4, 8, 16, 32, 64, 128, 0x7F, 0x80, 234, 0xF0]
     p = O.prefix(codes, r)
     v = p if r <= 4 else p << (8 - r)
+    lanes = _lane_words_of(codes)
     for gid in range(8):
         for tg in range(4):
-            words = _lane_words(codes, gid, tg)
+            words = lanes[(gid, tg)]
             for W in range(8):
                 regs = build_host(r, W, words)
                 halves = regs.view(np.uint16).view(np.float16).astype(np.float64).reshape(8, 2)
@@ -176,14 +159,14 @@ def test_operands_are_exact_prefix_values(build_host, r):
 
 
 def test_every_code_reaches_every_width(build_host):
-    # all 256 codes in the fields of one lane, block by block: the operand values take every
-    # prefix value exactly once per code
+    # 128 distinct codes in the fields of lane 0 (its share of the tile), high nibbles 0..15:
+    # every operand half decodes back to its own code's prefix
     codes = np.zeros((16, 256), dtype=np.int64)
     for w in range(8):
         for f in range(16):
             row, k = _field_coords(0, 0, w, f)
             codes[row, k] = 16 * (w + 8 * (f >= 8)) % 256 + (f & 15)
-    words = _lane_words(codes, 0, 0)
+    words = _lane_words_of(codes)[(0, 0)]
     for r in O.WIDTHS:
         seen = set()
         for W in range(8):
