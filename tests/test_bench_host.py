@@ -74,3 +74,12 @@ def test_copy_groups_cover_every_call_once_in_order():
     for sizes in ([5, 1, 1, 1, 9, 2], [1] * 7, [10]):
         flat = [i for g in bench.copy_groups(sizes, min_bytes=4) for i in g]
         assert flat == list(range(len(sizes)))
+
+
+def test_choose_case_cpu_baseline_is_bounded_and_well_formed():
+    t = bench.time.perf_counter()
+    rec = bench.cpu_choose_rate(budget_s=0.05, rows=1)
+    assert bench.time.perf_counter() - t < 30
+    assert rec["kind"] == "oracle" and rec["unit"] == "Gweights/s"
+    assert rec["value"] > 0 and rec["cores"] >= 1
+    assert "1 rows" in rec["sample"] and "pass" in rec["sample"]
