@@ -66,9 +66,12 @@ Readings where the pages are silent or ambiguous
 
 Parity status: every function here is pinned by tests under ``tests/``
 (``test_oracle_pins.py``) against worked examples printed on the pages,
-closed forms, invariants and brute force, except the end-to-end Mix'n'Match
-stack deviation, which is reported, not gated ("parity unpinned" beyond the
-per-layer, teacher-forced checks).
+closed forms, invariants and brute force.  ``ffn_block`` is pinned by a
+hand-worked two-row block (``tests/golden/ffn_block_hand.txt``) that a swapped
+gate and up, a skipped RMSNorm, a dropped residual, eps outside the square
+root or a transposed projection each fail.  Only the end-to-end Mix'n'Match
+stack deviation over many layers is reported, not gated ("parity unpinned"
+beyond the per-layer, teacher-forced checks).
 """
 
 from __future__ import annotations

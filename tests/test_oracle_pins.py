@@ -281,6 +281,56 @@ def test_ffn_block_zero_down_is_identity():
     assert np.array_equal(O.ffn_block(h, layer, 8, 128), h)
 
 
+def _ffn_golden(golden):
+    rows = golden("ffn_block_hand.txt")
+    eps = [float(r[1]) for r in rows if r[0] == "eps"][0]
+    h = np.array([[float(v) for v in r[1:]] for r in rows if r[0] == "h"])
+    out = np.array([[float(v) for v in r[1:]] for r in rows if r[0] == "out"])
+    layer = {}
+    for r in rows:
+        if r[0] == "codes":
+            n, k = int(r[2]), int(r[3])
+            q = np.array([int(v) for v in r[4:]], dtype=np.uint8).reshape(n, k)
+            layer[r[1]] = (q, np.ones((n, k), dtype=np.float16), np.ones((n, k), dtype=np.uint8))
+    return h, layer, eps, out
+
+
+def test_ffn_block_hand_example(golden):
+    """The block's result on a hand-worked two-row example (tests/golden/ffn_block_hand.txt)."""
+    h, layer, eps, out = _ffn_golden(golden)
+    got = O.ffn_block(h, layer, 8, 1, eps=eps)
+    assert np.allclose(got, out, rtol=0, atol=1e-13)
+
+
+def test_ffn_block_hand_example_catches_mutations(golden):
+    """Each plausible mistake in the block glue moves the hand-worked answer: swapped gate and
+    up, no RMSNorm, no residual, eps outside the square root, a transposed down projection."""
+    h, layer, eps, out = _ffn_golden(golden)
+
+    def lin(x, name, transpose=False):
+        q, s, z = layer[name]
+        if transpose:
+            q, s, z = q.T.copy(), s.T.copy(), z.T.copy()
+        return O.linear(x, q, s, z, 8, 1)
+
+    def block(swap=False, norm=True, residual=True, eps_outside=False, transpose_down=False):
+        if not norm:
+            n = h
+        elif eps_outside:
+            n = h / (np.sqrt(np.mean(h * h, axis=-1, keepdims=True)) + eps)
+        else:
+            n = O.rmsnorm(h, eps)
+        g, u = lin(n, "gate"), lin(n, "up")
+        a = O.silu(u) * g if swap else O.silu(g) * u
+        d = lin(a, "down", transpose=transpose_down)
+        return h + d if residual else d
+
+    assert np.allclose(block(), out, rtol=0, atol=1e-13)   # the reading itself matches
+    for kw in ({"swap": True}, {"norm": False}, {"residual": False}, {"eps_outside": True},
+               {"transpose_down": True}):
+        assert np.max(np.abs(block(**kw) - out)) > 1e-2, kw
+
+
 def test_mixnmatch_widths_recipe():
     w = synth.mixnmatch_widths(0)
     assert len(w) == 32 and sorted(w.tolist()) == [2] * 11 + [3] * 10 + [4] * 11
