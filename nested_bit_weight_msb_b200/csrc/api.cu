@@ -153,9 +153,10 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r, void* p
 
 size_t matq_linear_workspace(int M, int K, int N, int group) {
   if (M < 1 || N < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
-  // sized so that it also serves every smaller M (decode or prefill) with these K, N
+  // sized so that it also serves every smaller M with these K, N; a decode-size call keeps room
+  // for the prefill path's copy of x, which serves it when its activations do not fit the
+  // decode kernel's shared memory
   const size_t dec = decode_workspace_bytes(M <= kDecodeMaxM ? M : kDecodeMaxM);
-  if (M <= kDecodeMaxM) return dec;
   const size_t pre = workspace_header_bytes() + prefill_scratch_bytes(M, K);
   return pre > dec ? pre : dec;
 }
@@ -181,6 +182,15 @@ int matq_workspace_status(const void* workspace, int* status_out) {
   return MATQ_OK;
 }
 
+int matq_selftest_timeout(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace) return MATQ_ENULL;
+  if (!aligned16(workspace)) return MATQ_EALIGN;
+  if (ws_bytes < workspace_header_bytes()) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  return cuda_status(launch_wait_selftest((int*)workspace, MATQ_STATUS_SELFTEST, (cudaStream_t)stream));
+}
+
 int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
                 const uint8_t* zeros, int N, int r, int group, void* y, int y_mode, void* workspace,
                 size_t ws_bytes, void* stream) {
@@ -201,9 +211,10 @@ int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, con
   if (st) return st;
   const PlaneGeom g = make_geom(N, K);
   cudaError_t e;
+  e = cudaErrorNotSupported;
   if (M <= kDecodeMaxM)
     e = launch_decode(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
-  else
+  if (e == cudaErrorNotSupported)
     e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
   return cuda_status(e);
 }

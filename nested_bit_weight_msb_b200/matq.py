@@ -43,6 +43,7 @@ MATQ_OUT_F32_ACCUM = 2
 MATQ_OUT_SILU_GATED = 3
 MATQ_SLICE_TRUE_PREFIX = 0
 MATQ_SLICE_TRUNCATE = 1
+MATQ_STATUS_SELFTEST = 0x100
 
 WIDTHS = (2, 3, 4, 6, 8)
 DECODE_MAX_M = 16
@@ -61,6 +62,7 @@ _SIGNATURES = {
     "matq_linear_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "matq_workspace_init": (_c_int, [_c_vp, _c_size, _c_vp]),
     "matq_workspace_status": (_c_int, [_c_vp, ctypes.POINTER(_c_int)]),
+    "matq_selftest_timeout": (_c_int, [_c_vp, _c_size, _c_vp]),
     "matq_linear": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
     "matq_linear_noalloc": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
@@ -181,6 +183,13 @@ def workspace_status(ws) -> int:
     check(matq_workspace_status(_dev(ws, "workspace", _dt("uint8"), "workspace_status"), ctypes.byref(out)),
           "matq_workspace_status")
     return int(out.value)
+
+
+def selftest_timeout(ws, stream=None) -> None:
+    """Run the bounded-wait self-test on a workspace (its status then reports
+    MATQ_STATUS_SELFTEST, after about a second on the device)."""
+    check(matq_selftest_timeout(_dev(ws, "workspace", _dt("uint8"), "selftest_timeout"), ws.numel(),
+                                _stream_ptr(stream)), "matq_selftest_timeout")
 
 
 def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=None,
