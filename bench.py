@@ -43,6 +43,10 @@ import numpy as np
 WIDTHS = (2, 3, 4, 6, 8)
 D_MODEL, D_FF, GROUP = 4096, 14336, 128
 METRIC = "sliced r-bit linear: decode weight GB/s vs HBM peak; prefill TFLOP/s per r"
+# arithmetic each path computes in (not a precision claim): decode multiplies the exact fp16
+# weight levels with fp16 activations, prefill fp16 dequantised weight and activation tiles; both
+# accumulate in fp32
+DTYPES = {"GB/s": "f16-operands/f32-acc (bf16 in/out)", "TFLOP/s": "f16-operands/f32-acc (bf16 in/out)"}
 
 
 def parse():
@@ -51,9 +55,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="ffn8b_decode", choices=["ffn8b_decode", "ffn8b_prefill"])
+    ap.add_argument("--workload", default="ffn8b_decode",
+                    choices=["ffn8b_decode", "ffn8b_prefill", "stack32", "ffn9b_sweep", "linear1024"])
     ap.add_argument("--copies", type=int, default=6, help="device copies of the packed layer (L2 rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode workload only: leave out the prefill sub-record of the default line")
     ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose", "speedup"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
@@ -271,33 +278,53 @@ def fused_weights(w):
 # reference arm: the oracle on the host
 # ---------------------------------------------------------------------------------------------
 
+def reference_sampler(args, world):
+    """(sample(budget_s, rows) -> rate record, unit, config) of the oracle for a workload; the
+    config is the one our arm reports for the same workload."""
+    if args.workload == "stack32":
+        from nested_bit_weight_msb_b200 import synth
+        w = host_weights()
+        widths = [int(v) for v in synth.mixnmatch_widths(0, layers=STACK_LAYERS)]
+        return (lambda b, rows: cpu_stack_rate(w, budget_s=b, rows=min(rows, 128)), "GB/s",
+                stack_config(widths, world))
+    if args.workload in SWEEPS:
+        sw = SWEEPS[args.workload]
+        mats = sweep_mats(sw)
+        dec = [M for M in sw["batches"] if M <= 16]
+        return (lambda b, rows: cpu_sweep_rate(mats, sw["group"], dec, sw["widths"], budget_s=b, rows=min(rows, 128)),
+                "GB/s", sweep_config(args, sw, {k: list(v[0].shape) for k, v in mats.items()}, world))
+    spec = workload_spec(args.workload)
+    w = host_weights()
+    return (lambda b, rows: cpu_oracle_rate(spec, w, budget_s=b, rows=rows), spec["unit"],
+            workload_config(args, spec, world))
+
+
 def run_reference(args):
     world, rank, local = dist_setup()
     if rank != 0:
         return 0
-    spec = workload_spec(args.workload)
-    w = host_weights()
+    sample, unit, config = reference_sampler(args, world)
     # each step is a bounded sample, sized so that warm-up + steps stay within ~3 minutes
     budget = min(5.0, 150.0 / max(1, args.steps + args.warmup))
     rows = 256 if budget >= 2.0 else 32
     for _ in range(args.warmup):
-        cpu_oracle_rate(spec, w, budget_s=budget, rows=rows)
+        sample(budget, rows)
     vals = []
     for _ in range(args.steps):
-        vals.append(cpu_oracle_rate(spec, w, budget_s=budget, rows=rows))
+        vals.append(sample(budget, rows))
     v = float(np.mean([c["value"] for c in vals]))
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": spec["unit"], "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         # measured: the wall time of one step, i.e. of one bounded sample of the workload (value is
         # that sample's rate); a whole workload step on the oracle would take far longer
         "ms_per_step": float(np.mean([c["seconds"] for c in vals])) * 1e3,
         "step_is_bounded_sample": True,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(workload_config(args, spec, world), device="host cores (fp64 oracle)"),
+        "config": dict(config, device="host cores (fp64 oracle)"),
         "cpu_baseline": {"kind": "oracle", "cores": vals[0]["cores"], "sample": vals[0]["sample"], "value": v,
-                         "unit": spec["unit"]},
-        "e2e": {"value": v, "unit": spec["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                         "unit": unit},
+        "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -307,66 +334,118 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------------------------
 
-def run_ours(args):
-    import torch
-    world, rank, local = dist_setup()
-    maybe_init_pg(world, "nccl")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    from nested_bit_weight_msb_b200 import matq, synth
+class FfnBench:
+    """Device state of one workload's FFN step: the packed weights (rotating device copies), the
+    workload's activations, output buffers, a workspace, and the call helpers."""
 
-    spec = workload_spec(args.workload)
-    weights = host_weights()
-    # pack once per matrix (one-time), then clone into rotating copies
-    packed = {}
-    meta = {}
-    for name, (q, s, z) in fused_weights(weights).items():
-        dq = torch.from_numpy(q).to(dev)
-        p = matq.pack(dq, r_keep=8)
-        packed[name] = [p] + [p.clone() for _ in range(args.copies - 1)]
-        meta[name] = (torch.from_numpy(s.view(np.int16)).to(dev), torch.from_numpy(z).to(dev), q.shape[0], q.shape[1])
-        del dq
-    torch.cuda.synchronize()
+    def __init__(self, args, spec, packed, meta, dev, rank):
+        import torch
+        from nested_bit_weight_msb_b200 import matq, synth
+        self.args, self.spec, self.packed, self.meta, self.dev = args, spec, packed, meta, dev
+        self.matq = matq
+        self.batches = spec["batches"]
+        self.xs = {}
+        for M in self.batches:
+            xb, _ = synth.activations(M, D_MODEL, seed=rank, outlier_frac=spec["outlier"])
+            self.xs[M] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+        Mmax = max(self.batches)
+        self.ws = torch.zeros(max(matq.workspace_bytes(Mmax, K, N, GROUP) for _, (N, K) in FFN_CALLS),
+                              dtype=torch.uint8, device=dev)
+        self.gated = gated_epilogue(spec)
+        self.a_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in self.batches}
+        self.gu_buf = {M: torch.empty((M, out_cols(spec, "gate_up")), dtype=torch.bfloat16, device=dev)
+                       for M in self.batches}
+        self.y_buf = {M: torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev) for M in self.batches}
+        self.calls = [(r, M) for r in spec["widths"] for M in self.batches]
 
-    batches = spec["batches"]
-    xs = {}
-    for M in batches:
-        xb, _ = synth.activations(M, D_MODEL, seed=rank, outlier_frac=spec["outlier"])
-        xs[M] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
-    Mmax = max(batches)
-    ws = torch.zeros(max(matq.workspace_bytes(Mmax, K, N, GROUP) for _, (N, K) in FFN_CALLS),
-                     dtype=torch.uint8, device=dev)
-    a_buf = {M: torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev) for M in batches}
-    gated = gated_epilogue(spec)
-    gu_buf = {M: torch.empty((M, out_cols(spec, "gate_up")), dtype=torch.bfloat16, device=dev) for M in batches}
-    y_buf = {M: torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev) for M in batches}
+    def linear(self, name, copy, x, r, out):
+        s, z, N, K = self.meta[name]
+        mode = self.matq.MATQ_OUT_SILU_GATED if (name == "gate_up" and self.gated) else self.matq.MATQ_OUT_BF16
+        self.matq.linear(x, self.packed[name][copy], 8, s, z, N, r, GROUP, y=out, y_mode=mode, workspace=self.ws)
 
-    def linear(name, copy, x, r, out):
-        s, z, N, K = meta[name]
-        mode = matq.MATQ_OUT_SILU_GATED if (name == "gate_up" and gated) else matq.MATQ_OUT_BF16
-        matq.linear(x, packed[name][copy], 8, s, z, N, r, GROUP, y=out, y_mode=mode, workspace=ws)
-
-    def ffn(x, M, r, copy, y=None):
-        if gated:
-            linear("gate_up", copy, x, r, a_buf[M])
+    def ffn(self, x, M, r, copy, y=None):
+        if self.gated:
+            self.linear("gate_up", copy, x, r, self.a_buf[M])
         else:
-            linear("gate_up", copy, x, r, gu_buf[M])
-            matq.silu_mul_gu(gu_buf[M], out=a_buf[M])
-        linear("down", copy, a_buf[M], r, y_buf[M] if y is None else y)
+            self.linear("gate_up", copy, x, r, self.gu_buf[M])
+            self.matq.silu_mul_gu(self.gu_buf[M], out=self.a_buf[M])
+        self.linear("down", copy, self.a_buf[M], r, self.y_buf[M] if y is None else y)
 
-    calls = [(r, M) for r in spec["widths"] for M in batches]
+    def step(self, base=0):
+        for i, (r, M) in enumerate(self.calls):
+            self.ffn(self.xs[M], M, r, (base + i) % self.args.copies)
 
-    def step(base=0):
-        for i, (r, M) in enumerate(calls):
-            ffn(xs[M], M, r, (base + i) % args.copies)
 
-    stream = torch.cuda.Stream(device=dev)
+def graph_us_per_call(fn, stream, n=24):
+    """Device microseconds per call of fn(i) in steady state: a CUDA graph of n back-to-back calls
+    (rotating weight copies, so every call streams from HBM), median of 5 replays."""
+    import torch
     with torch.cuda.stream(stream):
-        step()
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = []
+        for _ in range(5):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            reps.append(e0.elapsed_time(e1) / n)
+    del g
+    return float(np.median(reps)) * 1e3
+
+
+def per_call_table(fb, stream):
+    """Per width and batch: each sliced-linear call of the FFN (gate+up with the gated epilogue,
+    down) timed on its own as back-to-back launches, with its roofline fraction (decode: GB/s of
+    algorithmic bytes over the measured HBM peak; prefill: TFLOP/s over the burst bf16 peak)."""
+    peaks = load_peaks()
+    rows = []
+    for r in fb.spec["widths"]:
+        for M in fb.batches:
+            row = {"r": r, "M": M}
+            tot_us = 0.0
+            for name, (N, K) in FFN_CALLS:
+                x = fb.xs[M] if name == "gate_up" else fb.a_buf[M]
+                out = fb.a_buf[M] if name == "gate_up" else fb.y_buf[M]
+                us = graph_us_per_call(lambda i: fb.linear(name, i % fb.args.copies, x, r, out), stream)
+                tot_us += us
+                if fb.spec["unit"] == "GB/s":
+                    b = linear_bytes(M, N, K, r, out_cols=out_cols(fb.spec, name))
+                    v = b / (us * 1e-6) / 1e9
+                    row[name] = {"us": round(us, 2), "GB/s": round(v, 1), "frac": round(v / peaks["hbm_gbs"], 3)}
+                else:
+                    v = 2 * M * N * K / (us * 1e-6) / 1e12
+                    row[name] = {"us": round(us, 2), "TFLOP/s": round(v, 1), "frac": round(v / peaks["bf16_tflops"], 3)}
+            if fb.spec["unit"] == "GB/s":
+                b = sum(linear_bytes(M, N, K, r, out_cols=out_cols(fb.spec, name)) for name, (N, K) in FFN_CALLS)
+                row["ffn"] = {"us": round(tot_us, 2), "GB/s": round(b / (tot_us * 1e-6) / 1e9, 1)}
+            else:
+                f = sum(2 * M * N * K for _, (N, K) in FFN_CALLS)
+                row["ffn"] = {"us": round(tot_us, 2), "TFLOP/s": round(f / (tot_us * 1e-6) / 1e12, 1)}
+            rows.append(row)
+    return rows
+
+
+def measure(args, spec, fb, stream, world, local, dev):
+    """Time the workload's step (device events around K graph replays after W warm-up replays,
+    max over ranks), then the dominant kernel's roofline, the per-call table and the end-to-end
+    step through the public calls with host buffers."""
+    import torch
+    with torch.cuda.stream(stream):
+        fb.step()
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
-            step()
+            fb.step()
         for _ in range(args.warmup):
             graph.replay()
         torch.cuda.synchronize()
@@ -383,44 +462,89 @@ def run_ours(args):
         barrier(world)
         torch.cuda.synchronize()
     # a timed run whose device-side waits ran out prints no number
-    st = matq.workspace_status(ws)
+    st = fb.matq.workspace_status(fb.ws)
     if st != 0:
         raise RuntimeError(f"device status {st} after the timed region: the timed calls did not complete normally")
     ms_total = max_over_ranks(world, e0.elapsed_time(e1), dev)
     ms_step = ms_total / args.steps
     b, f = step_units(spec)
     value = whole_job_value(spec["unit"], b, f, world, ms_step)
+    rl = roofline(args, spec, fb.linear, fb.xs, fb.a_buf if fb.gated else fb.gu_buf, stream, dev)
+    table = per_call_table(fb, stream)
+    e2e = end_to_end(args, spec, fb.ffn, fb.calls, fb.xs, fb.y_buf, stream, dev, world)
+    del graph
+    return {"value": value, "ms_per_step": ms_step, "roofline": rl, "per_r": table, "e2e": e2e,
+            "clocks": clk.summary(),
+            # per FFN: gated gate+up and down, one kernel each on the decode path, activation
+            # conversion + GEMM each on the prefill path
+            "gpu_launches": args.steps * len(fb.calls) * len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2)}
 
-    # ---- roofline of the dominant kernel: per-call device time of the sliced linear ----------
-    rl = roofline(args, spec, linear, xs, gu_buf, stream, dev)
 
-    # ---- end-to-end through the public API with host buffers --------------------------------
-    e2e = end_to_end(args, spec, ffn, calls, xs, y_buf, stream, dev, world)
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup()
+    maybe_init_pg(world, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from nested_bit_weight_msb_b200 import matq
 
-    line = None
+    spec = workload_spec(args.workload)
+    weights = host_weights()
+    # pack once per matrix (one-time), then clone into rotating copies
+    packed = {}
+    meta = {}
+    for name, (q, s, z) in fused_weights(weights).items():
+        dq = torch.from_numpy(q).to(dev)
+        p = matq.pack(dq, r_keep=8)
+        packed[name] = [p] + [p.clone() for _ in range(args.copies - 1)]
+        meta[name] = (torch.from_numpy(s.view(np.int16)).to(dev), torch.from_numpy(z).to(dev), q.shape[0], q.shape[1])
+        del dq
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device=dev)
+    res = measure(args, spec, FfnBench(args, spec, packed, meta, dev, rank), stream, world, local, dev)
+    # the default decode line also carries the prefill half of the metric (TFLOP/s per r)
+    pre = None
+    if args.workload == "ffn8b_decode" and not args.no_prefill:
+        pspec = workload_spec("ffn8b_prefill")
+        pfb = FfnBench(args, pspec, packed, meta, dev, rank)
+        pre = measure(args, pspec, pfb, stream, world, local, dev)
+        del pfb
+        torch.cuda.empty_cache()
+
     if rank == 0:
         peaks = load_peaks()
         line = {
-            "metric": METRIC, "value": value, "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16-operands/f32-acc (bf16 in/out)", "data": "synthetic",
+            "metric": METRIC, "value": res["value"], "unit": spec["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": DTYPES[spec["unit"]], "data": "synthetic",
             "config": dict(workload_config(args, spec, world),
                            l2=f"rotating {args.copies} device copies of the packed layer (> L2)",
                            timing="CUDA graph replay, CUDA events"),
-            "roofline": rl,
-            "e2e": e2e,
-            # per FFN: gated gate+up and down, one kernel each on the decode path, activation
-            # conversion + GEMM each on the prefill path
-            "gpu_launches": args.steps * len(calls) * len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2),
-            "clocks": clk.summary(),
+            "roofline": res["roofline"],
+            "e2e": res["e2e"],
+            "gpu_launches": res["gpu_launches"] + (pre["gpu_launches"] if pre else 0),
+            "clocks": res["clocks"],
             "peaks_source": peaks.get("_source"),
+            "per_r": res["per_r"],
         }
+        if pre is not None:
+            pspec = workload_spec("ffn8b_prefill")
+            line["prefill"] = {
+                "workload": "ffn8b_prefill", "value": pre["value"], "unit": pspec["unit"],
+                "ms_per_step": pre["ms_per_step"], "dtype": DTYPES[pspec["unit"]],
+                "config": dict(workload_config(argparse.Namespace(workload="ffn8b_prefill"), pspec, world),
+                               l2=f"rotating {args.copies} device copies of the packed layer (> L2)",
+                               timing="CUDA graph replay, CUDA events"),
+                "roofline": pre["roofline"], "e2e": pre["e2e"], "clocks": pre["clocks"], "per_r": pre["per_r"],
+                "gpu_launches": pre["gpu_launches"],
+            }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_oracle_rate(spec, weights)
+            if pre is not None:
+                line["prefill"]["cpu_baseline"] = cpu_oracle_rate(workload_spec("ffn8b_prefill"), weights)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graph
         dist.destroy_process_group()
     return 0
 
@@ -792,6 +916,433 @@ def run_speedup_case(args):
     return 0
 
 
+# ---------------------------------------------------------------------------------------------
+# the Mix'n'Match stack: 32 FFN layers of 8B shape, a width per layer
+# ---------------------------------------------------------------------------------------------
+STACK_LAYERS = 32
+STACK_BATCHES = (1, 16, 512)
+
+
+def stack_perms(layers=STACK_LAYERS):
+    """Seeded row permutations that make the stack's layers distinct matrices with the base
+    layer's statistics: gate/up by row pairs (a gate row stays next to its up row), down by rows."""
+    out = []
+    for l in range(layers):
+        rng = np.random.default_rng([7, l])
+        out.append((rng.permutation(D_FF), rng.permutation(D_MODEL)))
+    return out
+
+
+def stack_rows(perm_pairs):
+    return np.stack([2 * perm_pairs, 2 * perm_pairs + 1], axis=1).reshape(-1)
+
+
+def stack_layer_host(fused, perms, l):
+    """Host (codes, scales, zeros) of layer l's gate+up and down matrices."""
+    pp, pd = perms[l]
+    idx = stack_rows(pp)
+    return tuple(a[idx] for a in fused["gate_up"]), tuple(a[pd] for a in fused["down"])
+
+
+def stack_units(M, widths):
+    """(algorithmic bytes, flops) of one pass: per layer the gated gate+up call (bf16 in and out)
+    and the down call accumulating into the fp32 residual (read and written: 8 bytes per
+    element); the RMSNorm is not counted."""
+    b = f = 0
+    G = D_MODEL // GROUP
+    for r in widths:
+        b += linear_bytes(M, 2 * D_FF, D_MODEL, r, out_cols=D_FF)
+        b += D_MODEL * D_FF * r // 8 + D_MODEL * (D_FF // GROUP) * 3 + M * D_FF * 2 + M * D_MODEL * 8
+        f += 2 * M * (2 * D_FF * D_MODEL + D_MODEL * D_FF)
+    del G
+    return b, f
+
+
+class StackBench:
+    """Device state of the 32-layer stack: every layer packed keeping only its width's planes
+    (deployment mode A), the residual stream h (fp32), and the pass h <- h + FFN_l(RMSNorm(h))."""
+
+    def __init__(self, weights, dev, rank):
+        import torch
+        from nested_bit_weight_msb_b200 import matq, synth
+        self.matq = matq
+        self.widths = [int(w) for w in synth.mixnmatch_widths(0, layers=STACK_LAYERS)]
+        fused = fused_weights(weights)
+        perms = stack_perms()
+        q_gu = torch.from_numpy(fused["gate_up"][0]).to(dev)
+        s_gu = torch.from_numpy(fused["gate_up"][1].view(np.int16)).to(dev)
+        z_gu = torch.from_numpy(fused["gate_up"][2]).to(dev)
+        q_d = torch.from_numpy(fused["down"][0]).to(dev)
+        s_d = torch.from_numpy(fused["down"][1].view(np.int16)).to(dev)
+        z_d = torch.from_numpy(fused["down"][2]).to(dev)
+        self.layers = []
+        for l, r in enumerate(self.widths):
+            pp, pd = perms[l]
+            idx = torch.from_numpy(stack_rows(pp)).to(dev)
+            pdt = torch.from_numpy(pd).to(dev)
+            self.layers.append({
+                "r": r,
+                "gu": (matq.pack(q_gu.index_select(0, idx), r_keep=r), s_gu.index_select(0, idx).contiguous(),
+                       z_gu.index_select(0, idx).contiguous()),
+                "d": (matq.pack(q_d.index_select(0, pdt), r_keep=r), s_d.index_select(0, pdt).contiguous(),
+                      z_d.index_select(0, pdt).contiguous()),
+            })
+        del q_gu, q_d
+        self.h0, self.h, self.n, self.a = {}, {}, {}, {}
+        for M in STACK_BATCHES:
+            _, xv = synth.activations(M, D_MODEL, seed=rank, outlier_frac=0.01 if M > 16 else 0.0)
+            self.h0[M] = torch.from_numpy(np.ascontiguousarray(xv, dtype=np.float32)).to(dev)
+            self.h[M] = torch.empty((M, D_MODEL), dtype=torch.float32, device=dev)
+            self.n[M] = torch.empty((M, D_MODEL), dtype=torch.bfloat16, device=dev)
+            self.a[M] = torch.empty((M, D_FF), dtype=torch.bfloat16, device=dev)
+        Mmax = max(STACK_BATCHES)
+        self.ws = torch.zeros(max(matq.workspace_bytes(Mmax, K, N, GROUP) for _, (N, K) in FFN_CALLS),
+                              dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize()
+
+    def layer(self, lay, M, h):
+        m = self.matq
+        m.rmsnorm(h, eps=1e-5, out=self.n[M])
+        p, s, z = lay["gu"]
+        m.linear(self.n[M], p, lay["r"], s, z, 2 * D_FF, lay["r"], GROUP, y=self.a[M],
+                 y_mode=m.MATQ_OUT_SILU_GATED, workspace=self.ws)
+        p, s, z = lay["d"]
+        m.linear(self.a[M], p, lay["r"], s, z, D_MODEL, lay["r"], GROUP, y=h, y_mode=m.MATQ_OUT_F32_ACCUM,
+                 workspace=self.ws)
+
+    def run(self, M, h=None, h0=None):
+        """One pass through the 32 layers, starting from h0 (the batch's activations)."""
+        h = self.h[M] if h is None else h
+        h.copy_(self.h0[M] if h0 is None else h0)
+        for lay in self.layers:
+            self.layer(lay, M, h)
+
+
+def cpu_stack_rate(weights, budget_s=12.0, rows=128):
+    """The fp64 oracle on a bounded sample of the stack: the first `rows` rows of each matrix of
+    the first layers at M = 1, teacher-forced from N(0, 1) inputs; GB/s of algorithmic bytes."""
+    import oracle as O
+    from nested_bit_weight_msb_b200 import synth
+    fused = fused_weights(weights)
+    perms = stack_perms()
+    widths = synth.mixnmatch_widths(0, layers=STACK_LAYERS)
+    rng = np.random.default_rng(0)
+    done = 0.0
+    t0 = time.perf_counter()
+    n_layers = 0
+    while time.perf_counter() - t0 < budget_s or n_layers == 0:
+        l = n_layers % STACK_LAYERS
+        gu, d = stack_layer_host(fused, perms, l)
+        r = int(widths[l])
+        x = rng.standard_normal((1, D_MODEL))
+        O.gated_product(O.linear(x, gu[0][0:rows:2], gu[1][0:rows:2], gu[2][0:rows:2], r, GROUP),
+                        O.linear(x, gu[0][1:rows:2], gu[1][1:rows:2], gu[2][1:rows:2], r, GROUP))
+        O.linear(rng.standard_normal((1, D_FF)), d[0][:rows], d[1][:rows], d[2][:rows], r, GROUP)
+        done += linear_bytes(1, rows, D_MODEL, r) + linear_bytes(1, rows, D_FF, r)
+        n_layers += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt / 1e9, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"first {rows} rows of gate+up and down of {n_layers} stack layer(s) at M = 1, {dt:.1f} s",
+            "seconds": dt}
+
+
+def _oracle_cores():
+    cores = os.cpu_count()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=cores)
+    except Exception:
+        pass
+    return cores
+
+
+def stack_config(widths, world):
+    return {"workload": "stack32", "layers": STACK_LAYERS, "widths": list(widths),
+            "mean_bits": float(np.mean(widths)), "batches": list(STACK_BATCHES),
+            "shapes": "per layer: gate+up [28672,4096] (gated product in the epilogue), down [4096,14336] "
+                      "into the fp32 residual, group 128; layers are row-permuted copies of one seeded "
+                      "8B FFN layer, each packed with only its width's planes",
+            "parallelism": f"replicas x{world}", "l2": "32 distinct layers (2+ GB of planes) > L2",
+            "timing": "one CUDA graph per pass, CUDA events"}
+
+
+def run_stack(args):
+    """--workload stack32: the Mix'n'Match stack.  One step = one pass through the 32 layers at
+    each decode batch (M = 1 and 16), each pass one CUDA graph; the M = 512 pass (prefill path) is
+    timed the same way and reported beside it.  value = algorithmic bytes of the decode passes
+    over their device time."""
+    import torch
+    world, rank, local = dist_setup()
+    maybe_init_pg(world, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    weights = host_weights()
+    sb = StackBench(weights, dev, rank)
+    stream = torch.cuda.Stream(device=dev)
+    peaks = load_peaks()
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for M in STACK_BATCHES:
+            sb.run(M)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                sb.run(M)
+            graphs[M] = g
+        for _ in range(args.warmup):
+            for M in STACK_BATCHES:
+                graphs[M].replay()
+        torch.cuda.synchronize()
+    if sb.matq.workspace_status(sb.ws) != 0:
+        raise RuntimeError("device status after warm-up: the stack did not complete normally")
+    per_m = {}
+    clk = None
+    for M in STACK_BATCHES:
+        with torch.cuda.stream(stream):
+            barrier(world)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with ClockSampler(local) as c:
+                e0.record(stream)
+                for _ in range(args.steps):
+                    graphs[M].replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+            if M == 1:
+                clk = c.summary()
+        per_m[M] = max_over_ranks(world, e0.elapsed_time(e1), dev) / args.steps
+    if sb.matq.workspace_status(sb.ws) != 0:
+        raise RuntimeError("device status after the timed region: the stack did not complete normally")
+    dec = [M for M in STACK_BATCHES if M <= 16]
+    b_dec = sum(stack_units(M, sb.widths)[0] for M in dec)
+    ms_step = sum(per_m[M] for M in dec)
+    value = b_dec * world / (ms_step * 1e-3) / 1e9
+    table = []
+    for M in STACK_BATCHES:
+        b, f = stack_units(M, sb.widths)
+        row = {"M": M, "us": round(per_m[M] * 1e3, 1)}
+        if M <= 16:
+            v = b / (per_m[M] * 1e-3) / 1e9
+            row.update({"GB/s": round(v, 1), "frac": round(v / peaks["hbm_gbs"], 3)})
+        else:
+            v = f / (per_m[M] * 1e-3) / 1e12
+            row.update({"TFLOP/s": round(v, 1), "frac": round(v / peaks["bf16_tflops"], 3)})
+        table.append(row)
+    b1 = stack_units(1, sb.widths)[0]
+    ach = b1 / (per_m[1] * 1e-3) / 1e9
+    rl = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+          "traffic": None, "algorithmic_bytes": b1, "avg_us": per_m[1] * 1e3,
+          "kernel": "one 32-layer pass at M = 1 (per layer: RMSNorm, gated gate+up, down into the fp32 residual)",
+          "peak_source": peaks.get("_source")}
+    # end to end: the decode passes through the public calls, the batches' activations copied in
+    # from pinned host memory and the final residual streams copied back, every step
+    host_in = {M: sb.h0[M].cpu().pin_memory() for M in dec}
+    host_out = {M: torch.empty((M, D_MODEL), dtype=torch.float32).pin_memory() for M in dec}
+    dev_in = {M: torch.empty_like(sb.h0[M]) for M in dec}
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for M in dec:
+                dev_in[M].copy_(host_in[M], non_blocking=True)
+                sb.run(M, h0=dev_in[M])
+                host_out[M].copy_(sb.h[M], non_blocking=True)
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(world, e0.elapsed_time(e1), dev) / args.steps
+    for M in dec:
+        if not torch.equal(host_out[M].to(dev), sb.h[M]):
+            raise RuntimeError("end-to-end stack: the copied-back residual differs from the device one")
+    e2e = {"value": b_dec * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": sum(M * D_MODEL * 4 for M in dec), "d2h_bytes_per_step": sum(M * D_MODEL * 4 for M in dec),
+           "ms_per_step": ms_e2e}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": DTYPES["GB/s"], "data": "synthetic",
+            "config": stack_config(sb.widths, world),
+            "roofline": rl, "per_M": table, "e2e": e2e,
+            "gpu_launches": args.steps * sum(STACK_LAYERS * (3 if M <= 16 else 5) for M in dec),
+            "clocks": clk, "peaks_source": peaks.get("_source"),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_stack_rate(weights)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------
+# matrix sweeps: the Gemma-2-9B-shaped FFN over batch sizes, the 1024 x 1024 layer
+# ---------------------------------------------------------------------------------------------
+SWEEPS = {
+    "ffn9b_sweep": {"d_model": 3584, "d_ff": 14336, "group": 64, "batches": (1, 8, 32, 128, 512, 2048),
+                    "widths": WIDTHS, "ffn": True},
+    "linear1024": {"n": 1024, "k": 1024, "group": 128, "batches": (1,), "widths": WIDTHS, "ffn": False},
+}
+
+
+def sweep_mats(sw):
+    """Host (codes, scales, zeros) of a sweep's matrices: the 9B FFN's gate and up row-interleaved
+    into one gated matrix plus down, or the single 1024 x 1024 layer."""
+    from nested_bit_weight_msb_b200 import synth
+    g = sw["group"]
+    if sw["ffn"]:
+        d, f = sw["d_model"], sw["d_ff"]
+        w = {name: synth.parent_weights(N, K, g, seed=0, layer=0, proj=name)
+             for name, (N, K) in (("gate", (f, d)), ("up", (f, d)), ("down", (d, f)))}
+        return {"gate_up": tuple(interleave_rows(w["gate"][i], w["up"][i]) for i in range(3)), "down": w["down"]}
+    return {"linear": synth.parent_weights(sw["n"], sw["k"], g, seed=0, layer=0, proj="gate")}
+
+
+def sweep_config(args, sw, shapes, world):
+    return {"workload": args.workload, "group": sw["group"], "batches": list(sw["batches"]),
+            "widths": list(sw["widths"]), "shapes": shapes,
+            "parallelism": f"replicas x{world}", "l2": "rotating device copies of each pack (> 2x L2)",
+            "timing": "each call: CUDA graph of back-to-back launches, median of 5 replays"}
+
+
+def run_sweep(args):
+    """--workload ffn9b_sweep (Gemma-2-9B-shaped FFN: gate+up [28672, 3584] with the gated epilogue,
+    down [3584, 14336], group 64, M in {1, 8, 32, 128, 512, 2048}, every width, and the one-time
+    pack of each matrix) and --workload linear1024 (one 1024 x 1024 layer, group 128, M = 1, every
+    width).  Every sliced-linear call is timed on its own as back-to-back launches over rotating
+    weight copies (> 2x L2), with its roofline: decode batches (M <= 16) against the HBM copy peak,
+    larger ones against min(bf16 peak, arithmetic intensity x HBM peak).  value = algorithmic bytes
+    of the decode-batch calls over their device time."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq, synth
+    world, rank, local = dist_setup()
+    maybe_init_pg(world, "nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sw = SWEEPS[args.workload]
+    g = sw["group"]
+    peaks = load_peaks()
+    mats = sweep_mats(sw)
+    state = {}
+    for name, (q, sc, z) in mats.items():
+        N, K = q.shape
+        p0 = matq.pack(torch.from_numpy(q).to(dev), r_keep=8)
+        copies = int(min(256, max(2, (512 << 20) // p0.numel() + 1)))
+        state[name] = {"N": N, "K": K, "packs": [p0] + [p0.clone() for _ in range(copies - 1)],
+                       "s": torch.from_numpy(sc.view(np.int16)).to(dev), "z": torch.from_numpy(z).to(dev),
+                       "gated": name == "gate_up"}
+    Mmax = max(sw["batches"])
+    ws = torch.zeros(max(matq.workspace_bytes(Mmax, st["K"], st["N"], g) for st in state.values()),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    table, dec_b, dec_us = [], 0, 0.0
+    total_us = 0.0
+    with ClockSampler(local) as clk:
+        for M in sw["batches"]:
+            xs = {}
+            for name, st in state.items():
+                K = st["K"]
+                xb, _ = synth.activations(M, K, seed=rank, outlier_frac=0.01 if M > 16 else 0.0)
+                xs[name] = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+            for r in sw["widths"]:
+                row = {"M": M, "r": r}
+                for name, st in state.items():
+                    N, K = st["N"], st["K"]
+                    cols = N // 2 if st["gated"] else N
+                    y = torch.empty((M, cols), dtype=torch.bfloat16, device=dev)
+                    mode = matq.MATQ_OUT_SILU_GATED if st["gated"] else matq.MATQ_OUT_BF16
+                    n = len(st["packs"])
+                    us = graph_us_per_call(lambda i: matq.linear(xs[name], st["packs"][i % n], 8, st["s"], st["z"], N, r,
+                                                                 g, y=y, y_mode=mode, workspace=ws), stream,
+                                           n=min(n, 64))
+                    b = linear_bytes(M, N, K, r, group=g, out_cols=cols)
+                    fl = 2 * M * N * K
+                    gbs, tfs = b / (us * 1e-6) / 1e9, fl / (us * 1e-6) / 1e12
+                    if M <= 16:
+                        roof, frac = "hbm", gbs / peaks["hbm_gbs"]
+                        dec_b += b
+                        dec_us += us
+                    else:
+                        lim = min(peaks["bf16_tflops"], fl / b * peaks["hbm_gbs"] / 1e3)
+                        roof, frac = ("tensor" if lim == peaks["bf16_tflops"] else "hbm"), tfs / lim
+                    total_us += us
+                    row[name] = {"us": round(us, 2), "GB/s": round(gbs, 1), "TFLOP/s": round(tfs, 1),
+                                 "bound": roof, "frac": round(frac, 3)}
+                table.append(row)
+    if matq.workspace_status(ws) != 0:
+        raise RuntimeError("device status after the sweep: a call did not complete normally")
+    # the one-time pack of each matrix (all planes), 20 back-to-back packs over 3 code copies
+    pack = {}
+    if sw["ffn"]:
+        rng = np.random.default_rng(0)
+        for name, st in state.items():
+            N, K = st["N"], st["K"]
+            codes = [torch.from_numpy(rng.integers(0, 256, (N, K), dtype=np.uint8)).to(dev) for _ in range(3)]
+            planes = torch.empty(matq.matq_packed_bytes(N, K, 8), dtype=torch.uint8, device=dev)
+            us = graph_us_per_call(lambda i: matq.check(
+                matq.matq_pack(codes[i % 3].data_ptr(), N, K, 8, planes.data_ptr(), planes.numel(),
+                               torch.cuda.current_stream().cuda_stream), "matq_pack"), stream, n=20)
+            gbs = 2 * N * K / (us * 1e-6) / 1e9
+            pack[name] = {"N": N, "K": K, "us": round(us, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 3)}
+            del codes, planes
+    value = dec_b * world / (dec_us * 1e-6) / 1e9
+    first = table[0]
+    name0 = "gate_up" if sw["ffn"] else "linear"
+    dom = [r for r in table if r["M"] == min(sw["batches"]) and r["r"] == 2][0][name0]
+    rl = {"bound": "hbm", "achieved": dom["GB/s"], "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dom["frac"],
+          "traffic": None, "avg_us": dom["us"], "kernel": f"decode_kernel via matq_linear ({name0} r=2 M={first['M']})",
+          "peak_source": peaks.get("_source")}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": 1, "warmup": 3,
+            "ms_per_step": total_us / 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": DTYPES["GB/s"], "data": "synthetic",
+            "config": sweep_config(args, sw, {k: [v["N"], v["K"]] for k, v in state.items()}, world),
+            "roofline": rl, "per_call": table, "pack": pack, "clocks": clk.summary(),
+            "e2e": None, "e2e_note": "per-call sweep: the end-to-end form is measured on the FFN workloads",
+            "peaks_source": peaks.get("_source"),
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_sweep_rate(mats, g, [M for M in sw["batches"] if M <= 16], sw["widths"])
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def cpu_sweep_rate(mats, group, batches, widths, budget_s=12.0, rows=128):
+    """The fp64 oracle on a bounded sample of a sweep's decode calls: the first `rows` rows of each
+    matrix at every width and decode batch; GB/s of algorithmic bytes."""
+    import oracle as O
+    rng = np.random.default_rng(0)
+    done = 0.0
+    t0 = time.perf_counter()
+    passes = 0
+    while time.perf_counter() - t0 < budget_s or passes == 0:
+        for r in widths:
+            for M in batches:
+                for q, s, z in mats.values():
+                    K = q.shape[1]
+                    O.linear(rng.standard_normal((M, K)), q[:rows], s[:rows], z[:rows], r, group)
+                    done += linear_bytes(M, rows, K, r, group=group)
+        passes += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt / 1e9, "unit": "GB/s", "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"first {rows} rows of each matrix at every width and decode batch, {passes} pass(es), {dt:.1f} s",
+            "seconds": dt}
+
+
 def run_case(args):
     """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128,
     gated-product epilogue, as in the workloads) at width r and batch m, rotating through
@@ -832,6 +1383,10 @@ def main():
         return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "stack32":
+        return run_stack(args)
+    if args.workload in SWEEPS:
+        return run_sweep(args)
     return run_ours(args)
 
 

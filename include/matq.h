@@ -30,10 +30,10 @@
  *   - Shapes: N >= 1; K a positive multiple of 256 (matq_choose_codes: of group); M >= 1.
  *     group in {64, 128}.
  *   - Alignment: every device pointer must be 16-byte aligned.
- *   - Thread safety: calls on different streams may run concurrently; the only state is a
- *     thread-local "last CUDA error" and per-device caches of launch settings, except
- *     matq_linear_noalloc, whose calls on one device share a library-owned scratch array and
- *     must be ordered (see its contract).
+ *   - Thread safety: calls on different streams may run concurrently (with separate
+ *     workspaces); the only state is a thread-local "last CUDA error" and per-device caches of
+ *     launch settings, except matq_linear_noalloc, whose calls on one device share a
+ *     library-owned scratch array and must be ordered (see its contract).
  *
  * Packed plane layout ("MATQ-PL1"; written by matq_pack, read by every other call)
  *   The 8 code bits are split into five planes, most significant first:
@@ -138,16 +138,14 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r,
 /* ---- the sliced linear layer ----------------------------------------------------------- */
 
 /* Workspace bytes matq_linear needs for these sizes (a multiple of 256).
- * A workspace starts with a fixed 256-byte header holding the device status words (decode path
- * at byte 0, prefill path at byte 4).  The header must be zero-filled once before the first
- * call (matq_workspace_init, or any zero fill); a call that completes normally leaves it
- * unchanged, so a workspace is reused without re-initialisation.  The decode path (M <= 16)
- * needs nothing beyond the header; the prefill path keeps an fp16 copy of x after it, and the
- * size always leaves room for it (a decode-size call whose activations do not fit the decode
- * kernel's shared memory, e.g. M = 16 with K above about 24K, is served by the prefill path).  Calls
- * that share a workspace must be ordered on the device (one stream, or synchronised
- * streams).  A workspace sized for (M_max, K_max, N) serves every call with M <= M_max and
- * K <= K_max on either path. */
+ * A workspace starts with a fixed header (device status words and the ticket counters with
+ * which the CTAs sharing a split row group elect the one that adds their partial sums; no CTA
+ * waits for another).  The header must be zero-filled once before the first call
+ * (matq_workspace_init, or any zero fill); every call leaves the counters zero again, so a
+ * workspace is reused without re-initialisation.  Calls that share a workspace must be
+ * ordered on the device (one stream, or synchronised streams).  A workspace sized for
+ * (M_max, K_max, N) serves every call with M <= M_max and K <= K_max on either path
+ * (a decode-sized one serves prefill only for M <= 16). */
 size_t matq_linear_workspace(int M, int K, int N, int group);
 
 /* Zero the workspace header (asynchronous on `stream`).  ws_bytes: capacity of workspace. */
@@ -155,13 +153,16 @@ int matq_workspace_init(void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronously read the device status left in the workspace header: 0 if every earlier call
  * completed normally; otherwise the OR of the codes of device-side waits that ran out (each
- * wait gives up after about a second, records its code and lets the kernel return, so the
- * context stays usable).  The outputs of a call that recorded a code are undefined.  A non-zero
- * status stays until the header is zero-filled again (matq_workspace_init). */
+ * bounded wait gives up after about a second, records its code and lets the kernel return, so
+ * the context stays usable).  The outputs of a call that recorded a code are undefined, and a
+ * non-zero status requires matq_workspace_init before the workspace is used again. */
 int matq_workspace_status(const void* workspace, int* status_out);
 
 /* Status code recorded by matq_selftest_timeout. */
 #define MATQ_STATUS_SELFTEST 0x100
+/* Status code of a decode-path call (M <= 16) that met an activation with |x| >= 65536: the
+ * decode path multiplies in fp16, which has no such value; that call's y is undefined. */
+#define MATQ_STATUS_XRANGE 0x200
 
 /* Failure-detection self-test (asynchronous on `stream`): launches one warp that waits, with the
  * same bounded wait every libmatq kernel uses, on a shared-memory barrier that nothing ever
@@ -178,18 +179,22 @@ int matq_selftest_timeout(void* workspace, size_t ws_bytes, void* stream);
  *            the weight rows interleave the gate and up projections of an FFN (row 2i: gate
  *            row i, row 2i + 1: up row i); y is [M, N/2] bf16 with y[m, i] =
  *            bf16( silu(g) * u ), g and u the fp32 results of rows 2i and 2i + 1 (the gated
- *            product fused into the epilogue; silu(t) = t / (1 + exp(-t))).
- *            MATQ_OUT_F32_ACCUM adds the product to the fp32 values already in y.
+ *            product fused into the epilogue; silu(t) = t / (1 + exp(-t))).  MATQ_OUT_F32_ACCUM adds the
+ *            product to the fp32 values already in y.
  *   workspace device scratch of >= matq_linear_workspace(M, K, N, group) bytes, owned by
  *            the caller, header zero-filled once (see matq_workspace_init).
- * Kernel choice is internal: M <= 16 takes the decode path when its activations fit (planes streamed by bulk copies,
- * unpacked in registers into exact bf16 MMA operands, x used as it is (bf16), fp32
- * accumulation: no input value is rounded); larger M the prefill path (TMA-staged planes
- * dequantised to fp16 tiles in shared memory, tcgen05 MMA with TMEM accumulators).  The
- * prefill path rounds x and W_hat to fp16; it needs |x| and |W_hat| below 65504.  Kernels are
- * launched with programmatic dependent launch, so a call may start streaming weights while
- * the previous kernel in the stream finishes; it reads x and writes y only after that kernel
- * completes. */
+ * Kernel choice is internal: M <= 16 takes the decode path (persistent TMA-fed streaming
+ * kernel, weights unpacked in registers into exact fp16 MMA operands, fp32 accumulation;
+ * N <= 2^21); larger M the prefill path (TMA-staged planes dequantised to fp16 tiles in
+ * shared memory, tcgen05 MMA with TMEM accumulators).  Input range: the decode path converts
+ * x to fp16 operands, exact for |x| in [2^-14, 65504] (smaller values round to fp16's
+ * subnormal grid, 2^-24); an activation with |x| >= 65536 sets MATQ_STATUS_XRANGE in the
+ * workspace status and leaves that call's y undefined.  The prefill path divides each token's
+ * activations by the power of two that keeps its largest value finite in fp16 (exact) and
+ * multiplies the token's fp32 results back, so it serves any finite bf16 x; its fp16 weight
+ * tiles need |W_hat| below 65504.  Kernels are launched with programmatic
+ * dependent launch, so a call may start streaming weights while the previous kernel in the
+ * stream finishes; it reads x and writes y only after that kernel completes. */
 int matq_linear(const void* x, int M, int K,
                 const void* planes, int r_keep,
                 const uint16_t* scales, const uint8_t* zeros, int N,
@@ -221,9 +226,8 @@ int matq_linear(const void* x, int M, int K,
  *   no workspace arguments.
  * Limits: the sizes must fit the fixed scratch, i.e. matq_linear_workspace(M, K, N, group)
  * <= MATQ_NOALLOC_SCRATCH_BYTES; larger calls return MATQ_ESCRATCH and launch nothing.
- * The sizes fit while 256 + M*K*2 bytes (rounded up to 256) do: every M <= 16 with K below
- * 262,000, and e.g. M <= 1023 at K = 4096.  Use matq_linear with a caller workspace beyond
- * that.
+ * Every M <= 16 (decode path) fits; M > 16 (prefill path) fits while 262,400 + M*K*2 bytes
+ * (rounded up to 256) do, e.g. M <= 991 at K = 4096.  Use matq_linear with a caller workspace beyond that.
  * Set-up: the first call on each device, made with that device current, looks up the device
  * address of the array (cudaGetSymbolAddress; this can load libmatq's device code onto the
  * device) and caches it; a failure returns MATQ_ECUDA.  Make that first call before any

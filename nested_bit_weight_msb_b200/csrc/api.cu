@@ -153,10 +153,9 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r, void* p
 
 size_t matq_linear_workspace(int M, int K, int N, int group) {
   if (M < 1 || N < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
-  // sized so that it also serves every smaller M with these K, N; a decode-size call keeps room
-  // for the prefill path's copy of x, which serves it when its activations do not fit the
-  // decode kernel's shared memory
+  // sized so that it also serves every smaller M (decode or prefill) with these K, N
   const size_t dec = decode_workspace_bytes(M <= kDecodeMaxM ? M : kDecodeMaxM);
+  if (M <= kDecodeMaxM) return dec;
   const size_t pre = workspace_header_bytes() + prefill_scratch_bytes(M, K);
   return pre > dec ? pre : dec;
 }
@@ -211,10 +210,9 @@ int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, con
   if (st) return st;
   const PlaneGeom g = make_geom(N, K);
   cudaError_t e;
-  e = cudaErrorNotSupported;
   if (M <= kDecodeMaxM)
     e = launch_decode(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
-  if (e == cudaErrorNotSupported)
+  else
     e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
   return cuda_status(e);
 }

@@ -1,48 +1,48 @@
-// Decode path (M <= 16): a streaming sliced linear layer, bf16 mma.sync fed by a bulk-copy ring.
+// Decode path (M <= 16): one persistent, TMA-fed streaming kernel over the packed planes.
 //
 // Math ("MatGPTQ: Efficient and Accurate Inference over Nested Quantized Models", App. A.1:
 // delta folded into the zero point; §4: Y = X W_D computed as (W_D^T X^T)^T so that the
-// weights fill the 16-row MMA operand and the tokens the 8-column one).  Per group g of a row n:
+// weights fill the 16-row MMA operand and the tokens the 8-column one):
 //
-//   y[m, n] += s * ( 2^(8-r) * sum_{k in g} p[n,k] x[m,k] + (delta_r - z) * sum_{k in g} x[m,k] )
+//   y[m, n] = sum_g s[n,g] * ( 2^(8-r) * sum_{k in g} x[m,k] * p[n,k]
+//                              + (delta_r - z[n,g]) * sum_{k in g} x[m,k] )
 //
-// Operands.  A lane's plane words become bf16 A-operand registers in place (operands.cuh): a
-// mask-and-or against the bf16 pattern of 128 gives 128 + alpha_h * v exactly, v a field of at
-// most four bits and alpha_h a power of two fixed by the register's row half.  Widths 6 and 8 take
-// two MMAs per tile (code bits 7..4, then bits 3..2 or 3..0).  The activations are the B operand
-// as they are (bf16, loaded with ldmatrix): nothing is converted or rounded, so every bf16 input
-// value keeps its range and precision.  With D the MMA sum of a group and Ds = sum_k x[m,k]:
+// Operands.  A lane's plane words become fp16 A-operand registers in place: a mask-and-or
+// against the fp16 bit pattern of 1024 gives 1024 + sigma * v exactly (operands.cuh).  The
+// per-register powers of two sigma split into a per-row factor alpha (folded into the group
+// scale) and a per-input factor beta (inputs 8..15 of every 16-input MMA slice enter the B
+// operand divided by 16 for r <= 4, exact in fp16).  One more MMA per 16-input slice, with a
+// constant A operand (rows 0..7: -1024, rows 8..15: beta_k), accumulates both per-token sums
+// the algebra needs in registers: Dc = sum_k (-1024) * B_k (removes the 1024 bias) and
+// Ds = sum_k beta_k * B_k = sum_k x_k (the zero-point term).  Per slice of a group, in fp32:
 //
-//   y += a_main * D_main + a_lo * D_lo + s * (delta_r - z) * Ds,   a = s * (weight of the part) / alpha_h
+//   y += a_row * (D + Dc) + s * (delta_r - z) * Ds,   a_row = s * 2^(8-r) / alpha_row
 //
-// where each D starts the group at -128 * Ds (the C operand of the group's first MMA), so the
-// 128 bias cancels inside the MMA sum (a one-hot x gives D = alpha_h * v exactly).  Ds per
-// (token, group) is computed once per CTA with a constant-one MMA.
+// Everything is linear in the inputs, so a group may be split between warps.  No weight is
+// ever rounded; x's fp16 operand equals x except below 2^-14 (fp16 subnormals).
 //
-// Work split.  The row tiles (16 rows) are dealt to thread-block clusters in balanced contiguous
-// ranges; the Q CTAs of a cluster split the 256-input chunks (K) among themselves.  Inside a CTA
-// the work is a sequence of units (a group of RPW row tiles x one chunk; RPW = 2 for r <= 4, 1
-// above), tile-group-major.  A producer warp streams stage after stage of eight consecutive units
-// into a shared-memory ring (bulk copies of the planes of width r only: exactly r bits per weight
-// leave HBM; scales and zero points by cp.async), and the eight consumer warps take one unit of
-// each stage.  A warp accumulates a tile group over its consecutive units in registers; when a
-// tile group is complete the warps' partial sums are added in warp order (shared memory,
-// deterministic) and the result is written to y, or, with Q > 1, kept until the end of the
-// kernel, when the CTAs of the cluster add their results in rank order through distributed
-// shared memory.  No CTA ever waits on a CTA outside its cluster, and the cluster's CTAs are
-// co-scheduled by the hardware.  The activations of the CTA's K range stay resident in shared
-// memory for the whole kernel.
+// Schedule.  Work items are (row group of RG = 4 * RPW row tiles, 256-input chunk), ordered
+// row-group-major.  One persistent CTA per SM takes a balanced contiguous range of items
+// (stream-K style) and streams each into a shared-memory ring: the planes of width r (one
+// 2-D TMA per plane: exactly r bits per weight leave HBM), the chunk's bf16 activation rows
+// (one bulk copy per token into padded rows, so fragment loads are conflict-free) and the
+// rows' scales and zero points (cp.async).  Eight warps split each item 4 x 2: four row
+// slices of RPW row tiles times two 128-input slices; each warp reuses every activation
+// fragment across its row tiles.  Row groups inside a CTA's range are written directly.  A
+// row group split between CTAs is combined deterministically by whichever contributor finishes
+// it last: every contributor stores its partial sums in its workspace slot and takes a ticket
+// from the row group's counter; the one holding the last ticket adds the slots in CTA order and
+// resets the counter.  No CTA waits for another, so the result does not depend on which CTAs
+// are resident at the same time.  The counters live in the workspace header; every call leaves
+// them at zero.
 //
-// Launch.  Programmatic dependent launch: the kernel streams planes, scales and zero points
-// (which depend on no earlier kernel) as soon as it is resident, and waits for the preceding
-// kernel only before reading activations or writing y.  Every wait is bounded (~1 s): on a
-// timeout the kernel records a code in the workspace's status word and still reaches every
-// barrier, so it returns.
+// Launch.  Programmatic dependent launch: the kernel streams planes (which depend on no
+// earlier kernel) as soon as it is resident, and waits for the preceding kernel only before
+// reading activations or touching counters and y.
 #include <cuda.h>
+#include <cudaTypedefs.h>
 
-#include <map>
-#include <mutex>
-#include <tuple>
+#include <atomic>
 
 #include "../../include/matq.h"
 #include "common.cuh"
@@ -52,487 +52,533 @@
 
 namespace matq {
 
-constexpr int kDecConsumers = 8;                        // consumer warps (one unit of each stage each)
-constexpr int kDecThreads = 32 * (kDecConsumers + 1);   // and one producer warp
-constexpr int kDecMaxStages = 4;
-constexpr int kDecSmemBudget = 225 * 1024;
+constexpr int kRowSlices = 4;        // warps split an item's row tiles four ways ...
+// ... and its 256-input chunk into KSL = 2 slices of 128 inputs (8 warps, 256 threads: the
+// register budget of a thread stays at 255, and only two code variants share the I-cache)
+__host__ __device__ constexpr int k_slices(int NT) { return NT > 0 ? 2 : 2; }
+__host__ __device__ constexpr int dec_threads(int NT) { return 32 * kRowSlices * k_slices(NT); }
+// Resident CTAs per SM (CPS): two for M <= 8, r >= 6 on matrices with K <= 4096 (each CTA's 8
+// warps then fit 128 registers a thread, so an SM runs 16 warps and hides more latency; r = 6
+// and 8 carry the most operand-building work per item), otherwise one.  On long-K matrices a
+// row group would be split between too many CTAs; at r <= 4 the gain of the call is lost
+// because two resident CTAs keep the next kernel from starting its prologue early.
+constexpr int kMaxSMs = 160;  // bound on the SMs used, which sizes the partial-sum workspace
+__host__ __device__ constexpr int max_ctas_per_sm(int NT) { return NT == 1 ? 2 : 1; }
+constexpr int kXPitch = kChunk * 2 + 16;  // bytes per activation row in a stage (padded)
 
-__host__ __device__ constexpr int dec_rpw(int r) { return r <= 4 ? 2 : 1; }
-// bits of the planes in front of plane p: a stage holds plane p at 8 * RPW * 512 * this
-__host__ __device__ constexpr int dec_bits_before(int p) { return p == 0 ? 0 : p == 1 ? 2 : p == 2 ? 3 : p == 3 ? 4 : 6; }
-__host__ __device__ constexpr int dec_stage_planes(int r) { return 8 * dec_rpw(r) * 512 * r; }
-__host__ __device__ constexpr int dec_stage_bytes(int r) { return dec_stage_planes(r); }
+__host__ __device__ constexpr int rows_per_warp_tiles(int r) { return r <= 4 ? 4 : 2; }
 
 struct DecodeParams {
-  const uint8_t* planes;
-  unsigned long long poff[5];
+  int N, K, KC, RT, G, M, y_mode, C, NRG;
+  long long I;  // items
   const uint16_t* x;
   const uint16_t* scales;
   const uint8_t* zeros;
+  float* partial;
+  int* counters;
   void* y;
   int* err;
-  int N, K, KC, RT, G, M, y_mode;
-  int Q;       // CTAs per cluster; they split the chunks
-  int ncl;     // clusters; they split the row tiles
-  int S;       // ring depth
-  int xpitch;  // bytes per activation row in shared memory
-  int mspitch, mzpitch;  // bytes per row of the resident scales / zero points
-  int o_x, o_zero, o_ds, o_ms, o_mz, o_slots, o_cbuf, o_ring, o_bar;  // shared-memory layout
 };
 
-// Operand kinds and dequantisation constants of each width (see the file comment).
-template <int R>
-struct DecWidth {
-  static constexpr int kMain = R == 2 ? kOpP0 : R == 3 ? kOpNib3 : kOpNib4;
-  static constexpr bool kLo = R >= 6;
-  static constexpr int kLoKind = R == 6 ? kOpP3 : kOpNibLo;
-  static constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
-  __device__ static float a_main(int h) {
-    return (R <= 4 ? (float)(1 << (8 - R)) : 16.f) / (float)op_alpha(kMain, h);
-  }
-  __device__ static float a_lo(int h) { return kLo ? (R == 6 ? 4.f : 1.f) / (float)op_alpha(kLoKind, h) : 0.f; }
+template <int R, int NT, int GROUP, int CPS>
+struct DecodeLayout {
+  static constexpr int RPW = rows_per_warp_tiles(R);
+  static constexpr int RG = kRowSlices * RPW;           // row tiles per item
+  static constexpr int NG = kChunk / GROUP;             // groups per chunk
+  static constexpr int NTOK = NT * 8;
+  static constexpr int kPlanes = RG * R * 512;          // all planes of width r for the item
+  static constexpr int kX = NTOK * kXPitch;             // activation rows of the chunk
+  static constexpr int kMetaS = RG * 16 * 8;            // per row: up to 4 fp16 scales (8 B)
+  static constexpr int kMetaZ = RG * 16 * 4;            // per row: one aligned 4-byte word of zeros
+  static constexpr int oX = kPlanes;
+  static constexpr int oS = oX + kX;
+  static constexpr int oZ = oS + kMetaS;
+  static constexpr int kStage = ((oZ + kMetaZ) + 127) & ~127;
+  static constexpr int KSL = k_slices(NT);
+  static constexpr int kThreads = dec_threads(NT);
+  static constexpr int kRed = (KSL - 1) * kRowSlices * RPW * NT * 4 * 32 * 4;
+  // ring depth: up to 4 stages within the CTA's share of the SM's shared memory
+  static constexpr int kSmemBudget = CPS == 2 ? 113 * 1024 : 224 * 1024;
+  static constexpr int kStagesFit = (kSmemBudget - kRed - 256) / kStage;
+  static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit < 2 ? 2 : kStagesFit;
+  static constexpr int oRed = kStages * kStage;     // k-slice reduction buffer
+  static constexpr int oBar = oRed + kRed;
+  static constexpr int kSmem = oBar + 2 * kStages * 8 + 128;
+  static_assert(kSmem <= kSmemBudget, "decode stage ring exceeds the CTA's shared memory");
 };
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
+// plane p's offset inside an item's plane region (RG row tiles each)
+template <int RG>
+__device__ __forceinline__ int item_plane_off(int p) {
+  return RG * 512 * (p == 0 ? 0 : p == 1 ? 2 : p == 2 ? 3 : p == 3 ? 4 : 6);
+}
 
-// Scales (NG fp16, in NG / 2 words) and zero points (NG bytes) of the rows a consumer lane
-// touches in one unit (tile j, row half h).
-template <int RPW, int NG>
-struct DecMeta {
-  uint32_t s[RPW][2][NG / 2];
-  uint32_t z[RPW][2];
-};
-// from the CTA's resident scales [row][group] and zero points [row][group] (rows of the cluster's
-// tiles, groups of the CTA's chunks): unit of tile group p, chunk kcl
-template <int RPW, int NG>
-__device__ __forceinline__ void dec_meta_read(const DecodeParams& P, const uint8_t* smem, int p, int kcl, int lane,
-                                              DecMeta<RPW, NG>& m) {
-  const int gid = lane >> 2;
+// Lane words of the NB blocks NB*KS .. NB*KS+NB-1 of row tile t (at their natural indices).
+template <int R, int RG, int NB, int KS>
+__device__ __forceinline__ void lds_slice_words(const uint8_t* planes, int t, int lane, LaneWords& L) {
+  constexpr int w0 = NB * KS;                             // first block of the slice
+  constexpr int half = w0 / 4, wo = (w0 % 4) * 4;         // 2-bit planes: 512-byte half, byte offset
+  auto two_bit = [&](int p, uint32_t* dst) {
+    const uint8_t* src = planes + item_plane_off<RG>(p) + t * 1024 + half * 512 + lane * 16 + wo;
+    if constexpr (NB == 4) {
+      const uint4 a = *reinterpret_cast<const uint4*>(src);
+      dst[w0] = a.x; dst[w0 + 1] = a.y; dst[w0 + 2] = a.z; dst[w0 + 3] = a.w;
+    } else {
+      const uint2 a = *reinterpret_cast<const uint2*>(src);
+      dst[w0] = a.x; dst[w0 + 1] = a.y;
+    }
+  };
+  auto one_bit = [&](int p, uint32_t* dst) {
+    const uint8_t* src = planes + item_plane_off<RG>(p) + t * 512 + lane * 16 + (w0 / 2) * 4;
+    if constexpr (NB == 4) {
+      const uint2 a = *reinterpret_cast<const uint2*>(src);
+      dst[w0 / 2] = a.x; dst[w0 / 2 + 1] = a.y;
+    } else {
+      dst[w0 / 2] = *reinterpret_cast<const uint32_t*>(src);
+    }
+  };
+  two_bit(0, L.p0);
+  if constexpr (R >= 3) one_bit(1, L.p1);
+  if constexpr (R >= 4) one_bit(2, L.p2);
+  if constexpr (R >= 6) two_bit(3, L.p3);
+  if constexpr (R >= 8) two_bit(4, L.p4);
+}
+
+// B-operand registers of one 16-input MMA slice (inputs k0..k0+15 of the chunk) for token
+// tile nt, built from the bf16 activation rows in the stage: {x[k], x[k+1]} and
+// {x[k+8], x[k+9]} * hi_scale as fp16 pairs, k = k0 + 2*(lane%4), token 8*nt + lane/4.
+__device__ __forceinline__ void b_frag(const uint8_t* xs, int nt, int k0, int lane, float hi_scale, uint32_t& b0,
+                                       uint32_t& b1) {
+  const uint8_t* row = xs + (nt * 8 + (lane >> 2)) * kXPitch + (k0 + 2 * (lane & 3)) * 2;
+  const uint32_t lo = *reinterpret_cast<const uint32_t*>(row);
+  const uint32_t hi = *reinterpret_cast<const uint32_t*>(row + 16);
+  __half2 l = __floats2half2_rn(__uint_as_float(lo << 16), __uint_as_float(lo & 0xFFFF0000u));
+  __half2 h = __floats2half2_rn(__uint_as_float(hi << 16) * hi_scale, __uint_as_float(hi & 0xFFFF0000u) * hi_scale);
+  b0 = *reinterpret_cast<uint32_t*>(&l);
+  b1 = *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ long long item_begin(long long c, long long I, long long C) { return c * I / C; }
+// CTA whose range holds item u (every CTA has at least one item: C <= I)
+__device__ __forceinline__ long long item_owner(long long u, long long I, long long C) {
+  return ((u + 1) * C - 1) / I;
+}
+
+// Work of one warp: RPW row tiles (row slice rs) x input slice KS of every item.
+template <int R, int NT, int GROUP, int CPS, int KS, typename Refill>
+__device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                                            float* red, long long c, long long ib, long long ie, int rs, int lane,
+                                            Refill&& refill) {
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
+  constexpr int RPW = Lt::RPW, RG = Lt::RG, NG = Lt::NG, KSL = Lt::KSL;
+  constexpr int NB = 8 / KSL;                                    // 32-input blocks per slice
+  constexpr int kPromoteEvery = (GROUP / 32 < NB) ? GROUP / 32 : NB;  // blocks per scale group part
+  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
+  constexpr float kHiScale = (R <= 4) ? 0.0625f : 1.0f;
+  // constant A operands: -1024 everywhere (bias removal) and beta per input (token sums)
+  constexpr uint32_t kNeg1024 = 0xE400E400u;
+  constexpr uint32_t kOne = 0x3C003C00u, kBetaHi = (R <= 4) ? 0x4C004C00u : 0x3C003C00u;  // 1.0, 16.0
+  constexpr int kLaneFloats = RPW * NT * 4;
+  constexpr int kSlotFloats = kLaneFloats * 32;
+  const int gid = lane >> 2, tg = lane & 3;
+  const int nitems = (int)(ie - ib);
+  float amul[2];
+  if constexpr (R == 2) { amul[0] = 64.f; amul[1] = 16.f; }
+  else if constexpr (R == 3) { amul[0] = amul[1] = 32.f; }
+  else if constexpr (R == 4) { amul[0] = amul[1] = 16.f; }
+  else { amul[0] = amul[1] = 1.f; }
+  // One constant-A MMA yields both token sums: A rows 0..7 are -1024 (D rows 0..7 = Dc) and
+  // rows 8..15 are beta_k (D rows 8..15 = Ds).  Fragment registers: {row g, k lo}, {row g+8,
+  // k lo}, {row g, k hi}, {row g+8, k hi}; result {Dc(t), Dc(t+1), Ds(t), Ds(t+1)}.
+  const uint32_t Acs[4] = {kNeg1024, kOne, kNeg1024, kBetaHi};
+
+  float yacc[RPW][NT][4];
 #pragma unroll
   for (int j = 0; j < RPW; ++j)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = 16 * (p * RPW + j) + gid + 8 * h;
-      const uint8_t* ms = smem + P.o_ms + r * P.mspitch + kcl * NG * 2;
-      const uint8_t* mz = smem + P.o_mz + r * P.mzpitch + kcl * NG;
-      if constexpr (NG == 2) {
-        m.s[j][h][0] = *reinterpret_cast<const uint32_t*>(ms);
-        m.z[j][h] = *reinterpret_cast<const uint16_t*>(mz);
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(ms);
-        m.s[j][h][0] = v.x;
-        m.s[j][h][1] = v.y;
-        m.z[j][h] = *reinterpret_cast<const uint32_t*>(mz);
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
+
+  bool ok = true;
+  // largest bf16 magnitude seen in this warp's share of the activations (packed pairs): the
+  // fp16 operands hold |x| < 65536 only
+  uint32_t xmax = 0;
+  // (row group, chunk) of the current item, advanced item by item (no division in the loop)
+  const int rg_first = (int)(ib / P.KC);
+  int rg = rg_first, kc = (int)(ib - (long long)rg_first * P.KC);
+  for (int n = 0; n < nitems; ++n) {
+    const int s = n % Lt::kStages;
+    if (ok) ok = mbar_wait(&full[s], (n / Lt::kStages) & 1, P.err, 2);
+    if (ok) {
+      const uint8_t* st = smem + s * Lt::kStage;
+      // range check of the activations this item converts: the warps of k-slice KS split its
+      // tokens by row slice (every token of the slice is read by exactly one of them)
+      for (int t = rs; t < P.M && t < Lt::NTOK; t += kRowSlices) {
+        // inputs 128 * KS .. + 127 of the chunk (2 bytes each), 4 per lane
+        const uint2 w = *reinterpret_cast<const uint2*>(st + Lt::oX + t * kXPitch + KS * 256 + lane * 8);
+        xmax = __vmaxu2(xmax, __vmaxu2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu));
       }
-    }
-}
+      LaneWords L[RPW];
+#pragma unroll
+      for (int j = 0; j < RPW; ++j) lds_slice_words<R, RG, NB, KS>(st, rs * RPW + j, lane, L[j]);
 
-// One unit: NTILES (<= RPW) row tiles x one 256-input chunk, accumulated into yacc.
-//   st      the stage; slot: the unit's index in it (= the consumer warp)
-//   kcl     chunk index inside the CTA's K range; kc: global chunk index
-//   xaddr   per token tile: ldmatrix row address of this lane (shared::cta), and the byte step per
-//           input (2, or 0 for the zero row that stands in for tokens >= M)
-//   row0    global row of the unit's first row
-template <int R, int NT, int GROUP, int NTILES>
-__device__ __forceinline__ void dec_unit(const uint8_t* st, int slot, int kcl, const DecMeta<dec_rpw(R), kChunk / GROUP>& meta,
-                                         const uint32_t (&xaddr)[NT], const uint32_t (&xstep)[NT], const float* ds_s,
-                                         int lane, float (&yacc)[dec_rpw(R)][NT][4]) {
-  using Wd = DecWidth<R>;
-  constexpr int RPW = dec_rpw(R);
-  constexpr int NG = kChunk / GROUP;   // groups per chunk
-  constexpr int BPG = GROUP / 32;      // 32-input blocks per group
-  constexpr int NPL = planes_for_width(R);
-  constexpr int CH = (NT == 1 && !Wd::kLo) ? 2 : 1;  // independent MMA chains per (tile, token tile)
-  const int tg = lane & 3;
-
-  float d[NTILES][NT][CH][4], dl[NTILES][NT][4], dsv[NT][2];
+      float d[RPW][NT][4], dcs[NT][4];
+      auto zero_acc = [&]() {
 #pragma unroll
-  for (int hc = 0; hc < 2; ++hc) {
-    HalfWords Hw[NTILES];
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int j = 0; j < NTILES; ++j) {
-      auto two_bit = [&](int p, uint32_t* dst) {
-        const uint4 v = lds128(st + dec_bits_before(p) * 8 * RPW * 512 + (j * 8 + slot) * 1024 + hc * 512 + lane * 16);
-        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+          for (int i = 0; i < 4; ++i) {
+            dcs[nt][i] = 0.f;
+#pragma unroll
+            for (int j = 0; j < RPW; ++j) d[j][nt][i] = 0.f;
+          }
       };
-      auto one_bit = [&](int p, uint32_t* dst) {
-        const uint2 v = lds64(st + dec_bits_before(p) * 8 * RPW * 512 + (j * 8 + slot) * 512 + lane * 16 + hc * 8);
-        dst[0] = v.x; dst[1] = v.y;
-      };
-      two_bit(0, Hw[j].p0);
-      if constexpr (NPL >= 2) one_bit(1, Hw[j].p1);
-      if constexpr (NPL >= 3) one_bit(2, Hw[j].p2);
-      if constexpr (NPL >= 4) two_bit(3, Hw[j].p3);
-      if constexpr (NPL >= 5) two_bit(4, Hw[j].p4);
-    }
+      // Byte offset of this lane's zero points inside their 4-byte windows: the same for every
+      // row the lane touches in the item (the rows differ by multiples of 8, and 8 * G is a
+      // multiple of 4).
+      const int zoff = (int)(((unsigned)gid * (unsigned)P.G + (unsigned)kc * NG) & 3u);
+      const uint8_t* srow = st + Lt::oS + (rs * RPW * 16 + gid) * 8;
+      const uint8_t* zrow = st + Lt::oZ + (rs * RPW * 16 + gid) * 4 + zoff;
+      // fold the inputs accumulated so far (all in scale group gl) into the running sums.
+      // Rows >= N read stale scales and zero points; their sums are never stored.
+      auto promote = [&](int gl) {
 #pragma unroll
-    for (int wb = 0; wb < 4; ++wb) {
-      const int W = 4 * hc + wb;
-      if (W % BPG == 0) {
-        // a new group: its activation sums, and every accumulator starts at -128 * Ds
-        const int gq = W / BPG;
+        for (int j = 0; j < RPW; ++j) {
+          float a[2], cz[2];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const float2 v = *reinterpret_cast<const float2*>(ds_s + (kcl * NG + gq) * 16 + 8 * nt + 2 * tg);
-          dsv[nt][0] = v.x;
-          dsv[nt][1] = v.y;
-        }
-#pragma unroll
-        for (int j = 0; j < NTILES; ++j)
+          for (int h = 0; h < 2; ++h) {
+            const int rr = j * 16 + 8 * h;  // row offset inside the warp's row slice
+            const float sv = __half2float(*reinterpret_cast<const __half*>(srow + rr * 8 + gl * 2));
+            const float zv = (float)zrow[rr * 4 + gl];
+            a[h] = sv * amul[h];
+            cz[h] = sv * (kDelta - zv);
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float b = -128.f * dsv[nt][i & 1];
-              d[j][nt][0][i] = b;
-#pragma unroll
-              for (int c = 1; c < CH; ++c) d[j][nt][c][i] = 0.f;
-              dl[j][nt][i] = b;
-            }
-      }
-      uint32_t b[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        ldmatrix_x4(xaddr[nt] + xstep[nt] * (uint32_t)(kcl * kChunk + 32 * W), b[nt][0], b[nt][1], b[nt][2], b[nt][3]);
-#pragma unroll
-      for (int j = 0; j < NTILES; ++j) {
-        uint32_t A[2][4];
-        switch (wb) {
-          case 0: build_bf16<Wd::kMain, 0>(Hw[j], A); break;
-          case 1: build_bf16<Wd::kMain, 1>(Hw[j], A); break;
-          case 2: build_bf16<Wd::kMain, 2>(Hw[j], A); break;
-          default: build_bf16<Wd::kMain, 3>(Hw[j], A); break;
+            for (int i = 0; i < 4; ++i)
+              yacc[j][nt][i] = fmaf(cz[i >> 1], dcs[nt][2 + (i & 1)],
+                                    fmaf(a[i >> 1], d[j][nt][i] + dcs[nt][i & 1], yacc[j][nt][i]));
         }
+        zero_acc();
+      };
+      zero_acc();
+
+#pragma unroll
+      for (int wb = 0; wb < NB; ++wb) {
+        uint32_t b0[2][NT], b1[2][NT];
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_bf16(d[j][nt][jj % CH], A[jj], b[nt][2 * jj], b[nt][2 * jj + 1]);
-        if constexpr (Wd::kLo) {
-          switch (wb) {
-            case 0: build_bf16<Wd::kLoKind, 0>(Hw[j], A); break;
-            case 1: build_bf16<Wd::kLoKind, 1>(Hw[j], A); break;
-            case 2: build_bf16<Wd::kLoKind, 2>(Hw[j], A); break;
-            default: build_bf16<Wd::kLoKind, 3>(Hw[j], A); break;
+          for (int nt = 0; nt < NT; ++nt)
+            b_frag(st + Lt::oX, nt, (NB * KS + wb) * 32 + 16 * jj, lane, kHiScale, b0[jj][nt], b1[jj][nt]);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16(dcs[nt], Acs, b0[jj][nt], b1[jj][nt]);
           }
+#pragma unroll
+        for (int j = 0; j < RPW; ++j) {
+          uint32_t A[2][4];
+          build_slice_operands<R, NB * KS>(L[j], wb, A);
 #pragma unroll
           for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16(dl[j][nt], A[jj], b[nt][2 * jj], b[nt][2 * jj + 1]);
+            for (int nt = 0; nt < NT; ++nt) mma_f16(d[j][nt], A[jj], b0[jj][nt], b1[jj][nt]);
         }
-      }
-      if (W % BPG == BPG - 1) {
-        // fold the group into the running sums
-        const int gq = W / BPG;  // group inside the chunk
-#pragma unroll
-        for (int j = 0; j < NTILES; ++j)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t sbits = meta.s[j][h][gq >> 1] >> (16 * (gq & 1));
-            const float s = __half2float(__ushort_as_half((unsigned short)(sbits & 0xFFFFu)));
-            const float z = (float)((meta.z[j][h] >> (8 * gq)) & 0xFFu);
-            const float am = s * Wd::a_main(h);
-            const float al = s * Wd::a_lo(h);
-            const float c = s * (Wd::kDelta - z);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int i = 2 * h + e;
-                float dm = d[j][nt][0][i];
-                if constexpr (CH == 2) dm += d[j][nt][1][i];
-                float acc = fmaf(c, dsv[nt][e], yacc[j][nt][i]);
-                acc = fmaf(am, dm, acc);
-                if constexpr (Wd::kLo) acc = fmaf(al, dl[j][nt][i], acc);
-                yacc[j][nt][i] = acc;
-              }
-          }
+        if ((wb + 1) % kPromoteEvery == 0) promote(((NB * KS + wb) * 32) / GROUP);
       }
     }
-  }
-}
-
-// Write one fragment value of a finished tile group to y (all 32 lanes call this together with
-// the same k, so the gated mode can pair rows 2i and 2i + 1 across lanes 4 apart).
-template <int NT>
-__device__ __forceinline__ void dec_out(const DecodeParams& P, float v, int k, int row0, int ntiles, int lane) {
-  const int gid = lane >> 2, tg = lane & 3;
-  const int j = k / (NT * 4), nt = (k >> 2) % NT, i = k & 3;
-  const int row = row0 + 16 * j + gid + 8 * (i >> 1);
-  const int tok = 8 * nt + 2 * tg + (i & 1);
-  const bool valid = j < ntiles && row < P.N && tok < P.M;
-  if (P.y_mode == MATQ_OUT_SILU_GATED) {
-    const float u = __shfl_down_sync(0xffffffffu, v, 4);
-    if ((gid & 1) == 0 && valid)
-      reinterpret_cast<__nv_bfloat16*>(P.y)[(size_t)tok * (P.N >> 1) + (row >> 1)] =
-          __float2bfloat16_rn(__fdividef(v, 1.0f + __expf(-v)) * u);
-    return;
-  }
-  if (!valid) return;
-  const size_t o = (size_t)tok * P.N + row;
-  if (P.y_mode == MATQ_OUT_BF16) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
-  else if (P.y_mode == MATQ_OUT_F32) reinterpret_cast<float*>(P.y)[o] = v;
-  else reinterpret_cast<float*>(P.y)[o] += v;
-}
-
-template <int R, int NT, int GROUP>
-__global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeParams P) {
-  constexpr int RPW = dec_rpw(R);
-  constexpr int NG = kChunk / GROUP;
-  constexpr int NPL = planes_for_width(R);
-  constexpr int FR = RPW * NT * 4;  // fragment values per lane of a tile group
-  constexpr int kStage = dec_stage_bytes(R);
-
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P.o_bar);
-  uint64_t* empty = full + kDecMaxStages;
-  uint64_t* xbar = empty + kDecMaxStages;
-  uint8_t* ring = smem + P.o_ring;
-  float* ds_s = reinterpret_cast<float*>(smem + P.o_ds);
-  float* slots = reinterpret_cast<float*>(smem + P.o_slots);  // [2][8 warps][FR][32 lanes]
-  float* cbuf = reinterpret_cast<float*>(smem + P.o_cbuf);    // [tile group][FR][32 lanes]
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // this CTA's row tiles (its cluster's) and chunks
-  const int q = P.Q > 1 ? (int)cluster_rank() : 0;
-  const int cl = blockIdx.x / P.Q;
-  const int t0 = (int)((long long)P.RT * cl / P.ncl), t1 = (int)((long long)P.RT * (cl + 1) / P.ncl);
-  const int T = t1 - t0;
-  const int NP = (T + RPW - 1) / RPW;
-  const int kc0 = (int)((long long)P.KC * q / P.Q), kc1 = (int)((long long)P.KC * (q + 1) / P.Q);
-  const int KCc = kc1 - kc0;
-  const int U = NP * KCc;
-  const int NST = (U + kDecConsumers - 1) / kDecConsumers;
-  const int S = P.S;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);  // the producer's expect-tx arrival (+ the planes' bytes)
-      mbar_init(&empty[s], kDecConsumers);
-    }
-    mbar_init(xbar, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // the row that stands in for tokens >= M
-  if (threadIdx.x < 8) reinterpret_cast<uint32_t*>(smem + P.o_zero)[threadIdx.x] = 0u;
-  __syncthreads();
-  pdl_launch_dependents();
-
-  bool ok = true;
-  if (warp == kDecConsumers) {
-    // ---------------- producer warp ----------------
-    // planes of stage n (lane 0): bulk copies, the bytes announced on the stage's barrier
-    auto issue_planes = [&](int n) {
-      const int s = n % S;
-      uint8_t* st = ring + s * kStage;
-      const int u0 = n * kDecConsumers, u1 = min(u0 + kDecConsumers, U);
-      uint32_t bytes = 0;
-      for (int u = u0; u < u1;) {
-        const int p = u / KCc, ue = min(u1, (p + 1) * KCc);
-        bytes += (uint32_t)((ue - u) * min(RPW, T - p * RPW) * 512 * R);
-        u = ue;
-      }
-      mbar_expect_tx(&full[s], bytes);
-      for (int u = u0; u < u1;) {
-        const int p = u / KCc, ue = min(u1, (p + 1) * KCc);
-        const int kcs = kc0 + (u - p * KCc);
-        const int ntl = min(RPW, T - p * RPW);
-        for (int j = 0; j < ntl; ++j) {
-          const size_t rt = (size_t)(t0 + p * RPW + j);
-#pragma unroll
-          for (int pl = 0; pl < NPL; ++pl) {
-            const int b = plane_bits(pl);
-            bulk_load(st + dec_bits_before(pl) * 8 * RPW * 512 + (j * 8 + (u - u0)) * b * 512,
-                      P.planes + P.poff[pl] + (rt * P.KC + kcs) * b * 512, (uint32_t)((ue - u) * b * 512), &full[s]);
-          }
-        }
-        u = ue;
-      }
-    };
-    // the planes of the first stages depend on no earlier kernel
-    const int pre = min(S, NST);
-    if (lane == 0)
-      for (int n = 0; n < pre; ++n) issue_planes(n);
-    pdl_wait();  // activations (and y) belong to earlier kernels in the stream
-    if (lane == 0) mbar_expect_tx(xbar, (uint32_t)(P.M * KCc * kChunk * 2));
     __syncwarp();
-    for (int m = lane; m < P.M; m += 32)
-      bulk_load(smem + P.o_x + m * P.xpitch, P.x + (size_t)m * P.K + (size_t)kc0 * kChunk, (uint32_t)(KCc * kChunk * 2),
-                xbar);
-    for (int n = pre; n < NST; ++n) {
-      if (lane == 0) {
-        if (ok) ok = mbar_wait(&empty[n % S], ((n / S) - 1) & 1, P.err, 2);
-        if (ok) issue_planes(n);
-      }
-    }
-  } else {
-    // ---------------- consumer warps ----------------
-    const int gid = lane >> 2, tg = lane & 3;
-    {
-      // scales and zero points of the cluster's rows for this CTA's chunks, resident for the whole
-      // kernel (they depend on no earlier kernel); eight loads in flight per thread
-      const int rows = 16 * T;
-      const int sw = KCc * NG / 2;  // 4-byte words of scales per row
-      const int zw = KCc * NG / 2;  // 2-byte words of zero points per row
-      const int ct = threadIdx.x, nct = 32 * kDecConsumers;
-      const int total = rows * (sw + zw);
-      for (int base = 0; base < total; base += 8 * nct) {
-        uint32_t v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int idx = base + k * nct + ct;
-          v[k] = 0u;
-          if (idx < total) {
-            const int row = idx < rows * sw ? idx / sw : (idx - rows * sw) / zw;
-            const int grow = 16 * t0 + row;
-            if (grow < P.N) {
-              if (idx < rows * sw)
-                v[k] = __ldg(reinterpret_cast<const unsigned int*>(P.scales + (size_t)grow * P.G + (size_t)kc0 * NG) +
-                             (idx - row * sw));
-              else
-                v[k] = __ldg(reinterpret_cast<const unsigned short*>(P.zeros + (size_t)grow * P.G + (size_t)kc0 * NG) +
-                             (idx - rows * sw - row * zw));
-            }
-          }
+    if (lane == 0) mbar_arrive(&empty[s]);
+    // the streaming warps (0..7) refill this slot with item n + S once every warp released it
+    if (rs + kRowSlices * KS < 8 && n + Lt::kStages < nitems && ok) {
+      ok = mbar_wait(&empty[s], (n / Lt::kStages) & 1, P.err, 1);
+      if (ok) {
+        int rg2 = rg, kc2 = kc + Lt::kStages;
+        while (kc2 >= P.KC) {
+          kc2 -= P.KC;
+          ++rg2;
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int idx = base + k * nct + ct;
-          if (idx < total) {
-            if (idx < rows * sw) {
-              const int row = idx / sw;
-              *reinterpret_cast<uint32_t*>(smem + P.o_ms + row * P.mspitch + (idx - row * sw) * 4) = v[k];
-            } else {
-              const int row = (idx - rows * sw) / zw;
-              *reinterpret_cast<uint16_t*>(smem + P.o_mz + row * P.mzpitch + (idx - rows * sw - row * zw) * 2) =
-                  (uint16_t)v[k];
-            }
-          }
-        }
+        refill(n + Lt::kStages, rg2, kc2);
       }
     }
-    pdl_wait();
-    // ldmatrix row addresses: lane l reads row l % 8 (a token) of matrix l / 8 (inputs +8 each)
-    uint32_t xaddr[NT], xstep[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int tok = 8 * nt + (lane & 7);
-      if (tok < P.M) {
-        xaddr[nt] = smem_u32(smem + P.o_x + tok * P.xpitch + (lane >> 3) * 16);
-        xstep[nt] = 2;
-      } else {
-        xaddr[nt] = smem_u32(smem + P.o_zero);
-        xstep[nt] = 0;
-      }
-    }
-    ok = mbar_wait(xbar, 0, P.err, 4);
-    // Ds[group][token] = sum of the group's activations, with a constant-one A operand
-    if (ok) {
-      const uint32_t kOnes[4] = {0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u};  // bf16 1.0
-      for (int gl = warp; gl < KCc * NG; gl += kDecConsumers) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float dd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int blk = 0; blk < GROUP / 32; ++blk) {
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(xaddr[nt] + xstep[nt] * (uint32_t)(gl * GROUP + 32 * blk), b0, b1, b2, b3);
-            mma_bf16(dd, kOnes, b0, b1);
-            mma_bf16(dd, kOnes, b2, b3);
-          }
-          if (gid == 0) *reinterpret_cast<float2*>(ds_s + gl * 16 + 8 * nt + 2 * tg) = make_float2(dd[0], dd[1]);
-        }
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecConsumers) : "memory");
 
-    float yacc[RPW][NT][4];
+    // flush at the end of a row group (or of this CTA's range); all warps get here for the
+    // same items, so the four k-slices of a row slice meet at a named barrier
+    if (n == nitems - 1 || kc == P.KC - 1) {
+      const long long g0 = (long long)rg * P.KC, g1 = g0 + P.KC;
+      const bool whole = g0 >= ib && g1 <= ie;
+      if (KS > 0) {
+        float4* mine =
+            reinterpret_cast<float4*>(red + ((KS - 1) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
-    for (int j = 0; j < RPW; ++j)
+        for (int j = 0; j < RPW; ++j)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+          for (int nt = 0; nt < NT; ++nt)
+            mine[j * NT + nt] = make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
+      if (KS == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
-    auto flush = [&](int p) {
-      float* dst = slots + ((p & 1) * kDecConsumers + warp) * FR * 32 + lane;
+        for (int k2 = 0; k2 < KSL - 1; ++k2) {
+          const float4* o = reinterpret_cast<const float4*>(red + (k2 * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+#pragma unroll
+          for (int j = 0; j < RPW; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float4 v = o[j * NT + nt];
+              yacc[j][nt][0] += v.x;
+              yacc[j][nt][1] += v.y;
+              yacc[j][nt][2] += v.z;
+              yacc[j][nt][3] += v.w;
+            }
+        }
+        auto store_y = [&](int j, int nt, int i, float v) {
+          const int row = (rg * RG + rs * RPW + j) * 16 + gid + 8 * (i >> 1);
+          const int tok = nt * 8 + 2 * tg + (i & 1);
+          if (row < P.N && tok < P.M) {
+            const size_t o = (size_t)tok * P.N + row;
+            if (P.y_mode == 0) reinterpret_cast<__nv_bfloat16*>(P.y)[o] = __float2bfloat16_rn(v);
+            else if (P.y_mode == 1) reinterpret_cast<float*>(P.y)[o] = v;
+            else reinterpret_cast<float*>(P.y)[o] += v;
+          }
+        };
+        // Four values of one (row tile j, token tile nt) fragment; the whole warp calls this.
+        // Gated mode: even rows (gate) take the odd row below (up) from the lane 4 higher and
+        // write silu(gate) * up at column row / 2 of y [M, N/2].
+        auto store4 = [&](int j, int nt, float v0, float v1, float v2, float v3) {
+          if (P.y_mode == 3) {
+            const float vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float u = __shfl_down_sync(0xffffffffu, vv[i], 4);
+              const int row = (rg * RG + rs * RPW + j) * 16 + gid + 8 * (i >> 1);
+              const int tok = nt * 8 + 2 * tg + (i & 1);
+              if ((gid & 1) == 0 && row < P.N && tok < P.M)
+                reinterpret_cast<__nv_bfloat16*>(P.y)[(size_t)tok * (P.N >> 1) + (row >> 1)] =
+                    __float2bfloat16_rn(__fdividef(vv[i], 1.0f + __expf(-vv[i])) * u);
+            }
+            return;
+          }
+          store_y(j, nt, 0, v0);
+          store_y(j, nt, 1, v1);
+          store_y(j, nt, 2, v2);
+          store_y(j, nt, 3, v3);
+        };
+        if (whole) {
+#pragma unroll
+          for (int j = 0; j < RPW; ++j)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) store4(j, nt, yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
+        } else if (ok) {
+          // Split row group: every contributor stores its partial sums in its workspace slot and
+          // takes a ticket; the one that takes the last ticket adds all of them in CTA order
+          // (deterministic: its own part from registers, the others' from the slots), writes y
+          // and resets the counter.  No CTA ever waits for another.
+          const long long cf = item_owner(g0, P.I, P.C), cl = item_owner(g1 - 1, P.I, P.C);
+          int* cnt = &P.counters[rg * kRowSlices + rs];
+          {
+            const int side = (rg == rg_first) ? 0 : 1;
+            float4* mine = reinterpret_cast<float4*>(
+                P.partial + ((size_t)(c * 2 + side) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+#pragma unroll
+            for (int j = 0; j < RPW; ++j)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                __stcg(&mine[j * NT + nt], make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]));
+          }
+          __threadfence();  // release: the partial sums before the ticket
+          __syncwarp();
+          int ticket = 0;
+          if (lane == 0) {
+            ticket = atomicAdd(cnt, 1);
+            if (ticket == (int)(cl - cf)) {
+              __threadfence();  // acquire: every other contributor's partial sums (fence + ticket)
+              *reinterpret_cast<volatile int*>(cnt) = 0;  // leave the counter at zero for the next call
+            }
+          }
+          ticket = __shfl_sync(0xffffffffu, ticket, 0);
+          __syncwarp();  // orders the other lanes' loads after lane 0's acquire
+          if (ticket == (int)(cl - cf)) {
+            float4 acc[RPW * NT];
+#pragma unroll
+            for (int q = 0; q < RPW * NT; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // every contributor in CTA order; kU at a time so the loads overlap
+            constexpr int kU = CPS == 2 ? 1 : (RPW * NT >= 8) ? 2 : (16 / (RPW * NT));
+            for (long long c2 = cf; c2 <= cl; c2 += kU) {
+              float4 v[kU][RPW * NT];
+#pragma unroll
+              for (int u = 0; u < kU; ++u) {
+                const long long cc = c2 + u;
+                if (cc <= cl && cc != c) {
+                  const int side2 = (rg == (int)(item_begin(cc, P.I, P.C) / P.KC)) ? 0 : 1;
+                  const float4* src = reinterpret_cast<const float4*>(
+                      P.partial + ((size_t)(cc * 2 + side2) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+#pragma unroll
+                  for (int q = 0; q < RPW * NT; ++q) v[u][q] = __ldcg(&src[q]);
+                } else if (cc == c) {
+#pragma unroll
+                  for (int j = 0; j < RPW; ++j)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+                      v[u][j * NT + nt] = make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]);
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < kU; ++u)
+                if (c2 + u <= cl)
+#pragma unroll
+                  for (int q = 0; q < RPW * NT; ++q) {
+                    acc[q].x += v[u][q].x;
+                    acc[q].y += v[u][q].y;
+                    acc[q].z += v[u][q].z;
+                    acc[q].w += v[u][q].w;
+                  }
+            }
+#pragma unroll
+            for (int j = 0; j < RPW; ++j)
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                store4(j, nt, acc[j * NT + nt].x, acc[j * NT + nt].y, acc[j * NT + nt].z, acc[j * NT + nt].w);
+          }
+        }
+      }
+      // the reduction buffer may be overwritten only after the k-slice-0 warps have read it
+      asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
 #pragma unroll
       for (int j = 0; j < RPW; ++j)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            dst[((j * NT + nt) * 4 + i) * 32] = yacc[j][nt][i];
-            yacc[j][nt][i] = 0.f;
-          }
-    };
-
-    int cur = -1;
-    for (int n = 0; n < NST; ++n) {
-      const int s = n % S;
-      const int u = n * kDecConsumers + warp;
-      const bool has = u < U;
-      const int p = has ? u / KCc : -1;
-      if (ok) ok = mbar_wait(&full[s], (n / S) & 1, P.err, 1);
-      if (has && p != cur) {
-        if (cur >= 0) flush(cur);
-        cur = p;
-      }
-      if (has && ok) {
-        const int kcl = u - p * KCc;
-        const uint8_t* st = ring + s * kStage;
-        DecMeta<RPW, NG> meta;
-        dec_meta_read<RPW, NG>(P, smem, p, kcl, lane, meta);
-        if (RPW == 2 && T - p * RPW >= 2)
-          dec_unit<R, NT, GROUP, RPW>(st, warp, kcl, meta, xaddr, xstep, ds_s, lane, yacc);
-        else
-          dec_unit<R, NT, GROUP, 1>(st, warp, kcl, meta, xaddr, xstep, ds_s, lane, yacc);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-
-      // tile groups whose last unit is in this stage: add the warps' sums (warp order) and finish
-      const int plo = (n * kDecConsumers + KCc) / KCc - 1;
-      const int phi = min(NP - 1, (n * kDecConsumers + kDecConsumers) / KCc - 1);
-      for (int pc = plo; pc <= phi; ++pc) {
-        if (cur == pc) {
-          flush(pc);
-          cur = -1;
-        }
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecConsumers) : "memory");
-        const int row0 = 16 * (t0 + pc * RPW);
-        const int ntl = min(RPW, T - pc * RPW);
-        for (int k = warp; k < FR; k += kDecConsumers) {
-          float v = 0.f;
-          for (int w = 0; w < kDecConsumers; ++w) {
-            // warp w holds part of tile group pc iff one of its units u = w (mod 8) lies in it
-            const bool touched = KCc >= kDecConsumers || ((((w - pc * KCc) % kDecConsumers) + kDecConsumers) % kDecConsumers) < KCc;
-            if (touched) v += slots[(((pc & 1) * kDecConsumers + w) * FR + k) * 32 + lane];
-          }
-          if (P.Q == 1) dec_out<NT>(P, v, k, row0, ntl, lane);
-          else cbuf[(pc * FR + k) * 32 + lane] = v;
-        }
-        asm volatile("bar.sync 1, %0;" ::"r"(32 * kDecConsumers) : "memory");
-      }
+          for (int i = 0; i < 4; ++i) yacc[j][nt][i] = 0.f;
+    }
+    if (++kc == P.KC) {
+      kc = 0;
+      ++rg;
     }
   }
+  // an activation of magnitude >= 65536 (bf16 magnitude bits >= 0x4780) has no fp16 operand:
+  // the call's outputs are undefined and the status word says so
+  const uint32_t big = max(xmax >> 16, xmax & 0xFFFFu);
+  if (__any_sync(0xffffffffu, big >= 0x4780u) && lane == 0) atomicOr(P.err, MATQ_STATUS_XRANGE);
+}
 
-  if (P.Q > 1) {
-    // the cluster's CTAs add their tile-group sums in rank order; each finishes a share of them
-    cluster_sync_all();
-    if (warp < kDecConsumers) {
-      for (int pc = (int)((long long)NP * q / P.Q); pc < (int)((long long)NP * (q + 1) / P.Q); ++pc) {
-        const int row0 = 16 * (t0 + pc * RPW);
-        const int ntl = min(RPW, T - pc * RPW);
-        for (int k = warp; k < FR; k += kDecConsumers) {
-          const float* src = cbuf + (pc * FR + k) * 32 + lane;
-          float v = 0.f;
-          for (int rk = 0; rk < P.Q; ++rk) v += ld_dsmem_f32(dsmem_addr(src, (uint32_t)rk));
-          dec_out<NT>(P, v, k, row0, ntl, lane);
-        }
+template <int R, int NT, int GROUP, int CPS>
+__global__ void __launch_bounds__(dec_threads(NT), CPS)
+decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+              const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tm3,
+              const __grid_constant__ CUtensorMap tm4, const DecodeParams P) {
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
+  constexpr int RG = Lt::RG, NG = Lt::NG, NTOK = Lt::NTOK;
+  constexpr int kNumPlanes = planes_for_width(R);
+  constexpr int kThreads = Lt::kThreads;
+  constexpr int kStreamers = 256;  // threads of warps 0..7, which refill the ring
+
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lt::oBar);
+  uint64_t* empty = full + Lt::kStages;
+  float* red = reinterpret_cast<float*>(smem + Lt::oRed);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long c = blockIdx.x;
+  const long long ib = item_begin(c, P.I, P.C), ie = item_begin(c + 1, P.I, P.C);
+  const int nitems = (int)(ie - ib);
+  const CUtensorMap* maps[5] = {&tm0, &tm1, &tm2, &tm3, &tm4};
+  const int mrows = P.M < NTOK ? P.M : NTOK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Lt::kStages; ++s) {
+      mbar_init(&full[s], 1 + kStreamers);  // thread 0's arrival + one arrival per streamer
+      mbar_init(&empty[s], kThreads / 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // activation rows >= M stay zero in every stage (nothing is ever copied there)
+  for (int s = 0; s < Lt::kStages; ++s)
+    for (int i = threadIdx.x; i < (NTOK - mrows) * kXPitch / 4; i += kThreads)
+      reinterpret_cast<uint32_t*>(smem + s * Lt::kStage + Lt::oX + mrows * kXPitch)[i] = 0u;
+  __syncthreads();
+  // the next kernel in the stream may launch its prologue now
+  pdl_launch_dependents();
+
+  // Planes of item n into slot n % S (2-D TMA by thread 0): they depend on no earlier kernel.
+  auto stream_planes = [&](int n, int rg, int kc) {
+    if (threadIdx.x == 0) {
+      const int s = n % Lt::kStages;
+      uint8_t* st = smem + s * Lt::kStage;
+      mbar_expect_tx_only(&full[s], Lt::kPlanes + mrows * kChunk * 2);
+#pragma unroll
+      for (int p = 0; p < kNumPlanes; ++p)
+        tma_load_2d(st + item_plane_off<RG>(p), maps[p], kc * plane_bits(p) * 64, rg * RG, &full[s]);
+    }
+  };
+  // Activation rows of item n: a bulk copy per token (counted in the bytes expected above).
+  auto stream_x = [&](int n, int kc) {
+    const int s = n % Lt::kStages;
+    const int t = threadIdx.x;
+    if (t < mrows)
+      bulk_load(smem + s * Lt::kStage + Lt::oX + t * kXPitch, P.x + (size_t)t * P.K + (size_t)kc * kChunk,
+                kChunk * 2, &full[s]);
+  };
+  // Scales and zero points (cp.async, one row per streamer thread) of item n, and the
+  // streamers' arrivals; called by the streamer threads (warps 0..7) only.
+  auto stream_meta = [&](int n, int rg, int kc) {
+    const int s = n % Lt::kStages;
+    uint8_t* st = smem + s * Lt::kStage;
+    const int t = threadIdx.x;
+    // scales (NG fp16) and the aligned 4-byte word of zeros holding this chunk's NG bytes.
+    // The word never crosses the end of the zeros array except when its NG = 2 bytes are the
+    // array's last two and start a word; that row is copied with a plain 2-byte load.
+    const int row = rg * RG * 16 + t;
+    bool plain = false;
+    if (t < RG * 16 && row < P.N) {
+      const uint16_t* sp = P.scales + (size_t)row * P.G + (size_t)kc * NG;
+      if constexpr (NG == 2) cp_async4(st + Lt::oS + t * 8, sp);
+      else cp_async8(st + Lt::oS + t * 8, sp);
+      const size_t zi = (size_t)row * P.G + (size_t)kc * NG;
+      if ((zi & 3) == 0 && zi + 4 > (size_t)P.N * P.G) {
+        plain = true;
+        *reinterpret_cast<uint16_t*>(st + Lt::oZ + t * 4) = *reinterpret_cast<const uint16_t*>(P.zeros + zi);
+      } else {
+        cp_async4(st + Lt::oZ + t * 4, P.zeros + (zi & ~(size_t)3));
       }
     }
-    cluster_sync_all();
+    if (plain) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      mbar_arrive(&full[s]);  // a plain arrive releases the plain store too
+    } else {
+      cp_async_arrive_noinc(&full[s]);
+    }
+    if (t == 0) mbar_arrive(&full[s]);
+  };
+  auto refill = [&](int n, int rg, int kc) {
+    stream_planes(n, rg, kc);
+    stream_x(n, kc);
+    stream_meta(n, rg, kc);
+  };
+
+  // Prologue: the weights of the first S items (planes, scales, zero points) depend on no
+  // earlier kernel and are requested at once; the activations after the wait.
+  const int pre = nitems < Lt::kStages ? nitems : Lt::kStages;
+  const int rg0 = (int)(ib / P.KC), kc0 = (int)(ib - (long long)rg0 * P.KC);
+  for (int n = 0, rg = rg0, kc = kc0; n < pre; ++n) {
+    stream_planes(n, rg, kc);
+    stream_meta(n, rg, kc);
+    if (++kc == P.KC) { kc = 0; ++rg; }
   }
+  pdl_wait();  // activations, counters and y belong to earlier kernels in the stream
+  for (int n = 0, kc = kc0; n < pre; ++n) {
+    stream_x(n, kc);
+    if (++kc == P.KC) kc = 0;
+  }
+
+  const int rs = warp & 3, ks = warp >> 2;
+  static_assert(Lt::KSL == 2, "two input slices per item");
+  if (ks == 0) decode_warp<R, NT, GROUP, CPS, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+  else decode_warp<R, NT, GROUP, CPS, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
 }
 
 // Failure-detection self-test: one warp waits, with the bounded wait every kernel uses, on a
@@ -554,182 +600,98 @@ cudaError_t launch_wait_selftest(int* err, int code, cudaStream_t s) {
 }
 
 // ---- host side -----------------------------------------------------------------------------
-// Workspace: [header: device status words (decode at byte 0, prefill at byte 4)][prefill scratch].
-constexpr size_t kHeaderBytes = 256;
+// Workspace: [header: error word + split-row-group counters, zero-filled once by the caller
+// and left zero by every call][decode partial-sum slots | prefill scratch].
+constexpr size_t kHeaderCounters = size_t(1) << 16;
+constexpr size_t kHeaderBytes = 256 + kHeaderCounters * sizeof(int);
 
 size_t workspace_header_bytes() { return kHeaderBytes; }
-long long max_decode_rows() { return 1LL << 30; }
-size_t decode_workspace_bytes(int) { return kHeaderBytes; }
+long long max_decode_rows() { return (long long)(kHeaderCounters / kRowSlices) * 8 * kTileRows; }
 
-namespace {
-
-struct DecLayout {
-  int S, xpitch, mspitch, mzpitch, o_x, o_zero, o_ds, o_ms, o_mz, o_slots, o_cbuf, o_ring, o_bar, smem;
-};
-
-// Shared-memory layout for a CTA with up to KCc chunks and NP tile groups; false if it cannot hold
-// two stages.
-template <int R, int NT, int GROUP>
-bool dec_layout(int M, int KCc, int NP, int Q, DecLayout& L) {
-  constexpr int NG = kChunk / GROUP;
-  constexpr int RPW = dec_rpw(R), FR = RPW * NT * 4;
-  auto up = [](int v, int a) { return (v + a - 1) / a * a; };
-  L.xpitch = KCc * kChunk * 2 + 16;  // +16 B: ldmatrix rows fall in distinct banks
-  int o = 0;
-  L.o_x = o;
-  o = up(o + M * L.xpitch, 128);
-  L.o_zero = o;
-  o += 128;
-  L.o_ds = o;
-  o = up(o + KCc * NG * 16 * 4, 128);
-  L.mspitch = KCc * NG * 2;
-  L.mzpitch = up(KCc * NG, 4);
-  L.o_ms = o;
-  o = up(o + NP * RPW * 16 * L.mspitch, 128);
-  L.o_mz = o;
-  o = up(o + NP * RPW * 16 * L.mzpitch, 128);
-  L.o_slots = o;
-  o += 2 * kDecConsumers * FR * 32 * 4;
-  L.o_cbuf = o;
-  if (Q > 1) o += NP * FR * 32 * 4;
-  L.o_bar = o;
-  o = up(o + (2 * kDecMaxStages + 1) * 8, 1024);
-  L.o_ring = o;
-  const int room = kDecSmemBudget - o;
-  int S = room / dec_stage_bytes(R);
-  if (S > kDecMaxStages) S = kDecMaxStages;
-  if (S < 2) return false;
-  L.S = S;
-  L.smem = o + S * dec_stage_bytes(R);
-  return true;
+size_t decode_workspace_bytes(int M) {
+  const int NT = (M <= 8) ? 1 : 2;
+  const size_t partial =
+      (size_t)2 * kMaxSMs * max_ctas_per_sm(NT) * kRowSlices * 4 * NT * 4 * 32 * sizeof(float);
+  return kHeaderBytes + ((partial + 255) & ~size_t(255));
 }
 
-// Clusters of Q CTAs (with this much shared memory) that can be resident at once, per device.
-int max_clusters(const void* kern, int Q, int smem, int sms) {
-  static std::mutex mu;
-  static std::map<std::tuple<int, const void*, int, int>, int> cache;
-  const int dev = current_device();
-  const auto key = std::make_tuple(dev, kern, Q, smem);
-  {
-    std::lock_guard<std::mutex> g(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) return it->second;
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
   }
-  int n = 0;
-  if (Q == 1) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, smem) != cudaSuccess) per_sm = 0;
-    n = per_sm * sms;
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(Q * sms);
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = Q;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();  // a failed query is not an error of the call
-  std::lock_guard<std::mutex> g(mu);
-  cache[key] = n;
-  return n;
+  return fn;
 }
 
-template <int R, int NT, int GROUP>
-cudaError_t launch_decode_t(DecodeParams P, int sms, cudaStream_t s) {
-  auto kern = decode_kernel<R, NT, GROUP>;
-  static std::mutex mu;
-  static unsigned long long attr_set = 0;  // devices whose shared-memory attribute is set
-  const int dev = current_device();
-  {
-    std::lock_guard<std::mutex> g(mu);
-    if (dev >= 64 || !(attr_set & (1ull << dev))) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemBudget);
+static cudaError_t plane_map(CUtensorMap* m, const uint8_t* base, const PlaneGeom& g, int p, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const int b = plane_bits(p);
+  const cuuint64_t dims[2] = {(cuuint64_t)g.KC * b * 64, (cuuint64_t)g.RT};
+  const cuuint64_t strides[1] = {(cuuint64_t)g.KC * b * 512};
+  const cuuint32_t box[2] = {(cuuint32_t)(b * 64), (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(base + g.off[p]), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int R, int NT, int GROUP, int CPS>
+static cudaError_t launch_decode_t(const uint8_t* planes, const PlaneGeom& g, DecodeParams P, int sms,
+                                   cudaStream_t s) {
+  using Lt = DecodeLayout<R, NT, GROUP, CPS>;
+  CUtensorMap maps[5];
+  for (int p = 0; p < 5; ++p) {
+    if (p < planes_for_width(R)) {
+      cudaError_t e = plane_map(&maps[p], planes, g, p, Lt::RG);
       if (e != cudaSuccess) return e;
-      if (dev < 64) attr_set |= 1ull << dev;
+    } else {
+      maps[p] = maps[0];
     }
   }
-  // Choose Q (CTAs per cluster splitting K): the smallest per-CTA share of the work
-  // (row tiles x chunks, a two-stage ring counted 15% slower) among the layouts that fit, fewer
-  // CTAs per cluster on a tie.  None fits when the CTA's activations cannot stay resident even
-  // at Q = 8: the caller then takes another path.
-  int bestQ = 0, best_ncl = 0;
-  long long best_cost = 0;
-  DecLayout best{};
-  for (int Q = 1; Q <= 8 && Q <= P.KC; Q *= 2) {
-    const int KCc = (P.KC + Q - 1) / Q;
-    DecLayout L;
-    // tile groups per cluster are bounded after the cluster count is known; size for the worst
-    int ncl_try = sms / Q;
-    if (ncl_try < 1) ncl_try = 1;
-    if (ncl_try > P.RT) ncl_try = P.RT;
-    int tiles = (P.RT + ncl_try - 1) / ncl_try;
-    if (!dec_layout<R, NT, GROUP>(P.M, KCc, (tiles + dec_rpw(R) - 1) / dec_rpw(R), Q, L)) continue;
-    int ncl = max_clusters((const void*)kern, Q, L.smem, sms);
-    if (ncl < 1) continue;
-    if (ncl > P.RT) ncl = P.RT;
-    if (ncl != ncl_try) {
-      tiles = (P.RT + ncl - 1) / ncl;
-      if (!dec_layout<R, NT, GROUP>(P.M, KCc, (tiles + dec_rpw(R) - 1) / dec_rpw(R), Q, L)) continue;
-    }
-    const long long cost = (long long)tiles * KCc * (L.S >= 3 ? 20 : 23);
-    if (bestQ == 0 || cost < best_cost) {
-      bestQ = Q;
-      best_cost = cost;
-      best_ncl = ncl;
-      best = L;
-    }
+  P.NRG = (g.RT + Lt::RG - 1) / Lt::RG;
+  P.I = (long long)P.NRG * g.KC;
+  const long long ctas = (long long)sms * CPS;
+  P.C = (int)(P.I < ctas ? P.I : ctas);
+  auto kern = decode_kernel<R, NT, GROUP, CPS>;
+  // the shared-memory attribute is set once per device for this kernel
+  static std::atomic<unsigned long long> attr_set{0};
+  const int dev = current_device();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (dev >= 64 || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lt::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(bit, std::memory_order_relaxed);
   }
-  if (bestQ == 0) return cudaErrorNotSupported;
-  P.Q = bestQ;
-  P.ncl = best_ncl;
-  P.S = best.S;
-  P.xpitch = best.xpitch;
-  P.o_x = best.o_x;
-  P.o_zero = best.o_zero;
-  P.o_ds = best.o_ds;
-  P.o_ms = best.o_ms;
-  P.o_mz = best.o_mz;
-  P.mspitch = best.mspitch;
-  P.mzpitch = best.mzpitch;
-  P.o_slots = best.o_slots;
-  P.o_cbuf = best.o_cbuf;
-  P.o_ring = best.o_ring;
-  P.o_bar = best.o_bar;
-  return launch_pdl_cluster(kern, dim3(best_ncl * bestQ), dim3(kDecThreads), (size_t)best.smem, bestQ, s, P);
+  return launch_pdl(kern, dim3(P.C), dim3(Lt::kThreads), (size_t)Lt::kSmem, s, maps[0], maps[1], maps[2], maps[3],
+                    maps[4], P);
 }
 
-template <int NT, int GROUP>
-cudaError_t launch_decode_r(int r, const DecodeParams& P, int sms, cudaStream_t s) {
+template <int NT, int GROUP, int CPS>
+static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom& g, const DecodeParams& P, int sms,
+                                   cudaStream_t s) {
   switch (r) {
-    case 2: return launch_decode_t<2, NT, GROUP>(P, sms, s);
-    case 3: return launch_decode_t<3, NT, GROUP>(P, sms, s);
-    case 4: return launch_decode_t<4, NT, GROUP>(P, sms, s);
-    case 6: return launch_decode_t<6, NT, GROUP>(P, sms, s);
-    default: return launch_decode_t<8, NT, GROUP>(P, sms, s);
+    case 2: return launch_decode_t<2, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 3: return launch_decode_t<3, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 4: return launch_decode_t<4, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 6: return launch_decode_t<6, NT, GROUP, CPS>(planes, g, P, sms, s);
+    default: return launch_decode_t<8, NT, GROUP, CPS>(planes, g, P, sms, s);
   }
 }
-
-}  // namespace
 
 cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g, const uint16_t* scales,
                           const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
                           cudaStream_t s) {
   const int NT = (M <= 8) ? 1 : 2;
-  const int sms = sm_count(current_device());
-  DecodeParams P{};
-  P.planes = (const uint8_t*)planes;
-  for (int p = 0; p < kPlanes; ++p) P.poff[p] = g.off[p];
-  P.x = (const uint16_t*)x;
-  P.scales = scales;
-  P.zeros = zeros;
-  P.y = y;
-  P.err = (int*)workspace;
+  uint8_t* ws = (uint8_t*)workspace;
+  int sms = sm_count(current_device());
+  if (sms > kMaxSMs) sms = kMaxSMs;
+  DecodeParams P;
   P.N = g.N;
   P.K = K;
   P.KC = g.KC;
@@ -737,8 +699,19 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
   P.G = K / group;
   P.M = M;
   P.y_mode = y_mode;
-  if (NT == 1) return group == 64 ? launch_decode_r<1, 64>(r, P, sms, s) : launch_decode_r<1, 128>(r, P, sms, s);
-  return group == 64 ? launch_decode_r<2, 64>(r, P, sms, s) : launch_decode_r<2, 128>(r, P, sms, s);
+  P.x = (const uint16_t*)x;
+  P.scales = scales;
+  P.zeros = zeros;
+  P.err = (int*)ws;
+  P.counters = (int*)(ws + 256);
+  P.partial = (float*)(ws + kHeaderBytes);
+  P.y = y;
+  const uint8_t* pl = (const uint8_t*)planes;
+  if (NT == 1 && g.KC <= 16)
+    return group == 64 ? launch_decode_r<1, 64, 2>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 2>(r, pl, g, P, sms, s);
+  if (NT == 1)
+    return group == 64 ? launch_decode_r<1, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 1>(r, pl, g, P, sms, s);
+  return group == 64 ? launch_decode_r<2, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<2, 128, 1>(r, pl, g, P, sms, s);
 }
 
 }  // namespace matq

@@ -9,15 +9,13 @@ namespace matq {
 cudaError_t launch_pack(const uint8_t* codes, const PlaneGeom& g, int r_keep, void* planes, cudaStream_t s);
 cudaError_t launch_slice(const void* planes, const PlaneGeom& g, int r, uint8_t* out, cudaStream_t s);
 
-// Workspace = [header: device status words (decode at byte 0, prefill at byte 4); zero-filled
-// once by the caller][scratch of the path taken].
+// Workspace = [header: device error words + split-row-group counters; zero-filled once by the
+// caller, left zero by every call][scratch of the path taken].
 size_t workspace_header_bytes();
 long long max_decode_rows();
 size_t decode_workspace_bytes(int M);  // header included
 // Bounded-wait self-test: a kernel whose wait runs out ORs `code` into *err and returns.
 cudaError_t launch_wait_selftest(int* err, int code, cudaStream_t s);
-// cudaErrorNotSupported (nothing launched): the activations of these sizes cannot stay resident
-// in the decode kernel's shared memory; the prefill path serves the call instead.
 cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
                           const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
                           int y_mode, void* workspace, cudaStream_t s);

@@ -124,98 +124,6 @@ __device__ __forceinline__ void build_operands(const LaneWords& L, uint32_t (&A)
   }
 }
 
-// ---- bf16 operands (decode path) ------------------------------------------------------------
-// Every bf16 half is 128 + alpha * v exactly: a mask-and-or against the bf16 bit pattern of 128
-// (exponent 7, seven mantissa bits of step 1) places a field of at most 7 bits in the mantissa.
-// alpha depends only on the register's row half h = rho & 1, never on its input half, so the
-// activations enter the B operand unscaled (raw bf16).  Fields wider than 4 bits never occur:
-// widths 6 and 8 are served as a high part (code bits 7..4) plus a low part (bits 3..2 or 3..0),
-// one MMA each.
-//
-// Plane words of one lane for half a chunk (blocks 4*hc .. 4*hc + 3, 128 inputs): 2-bit planes
-// one word per block, 1-bit planes one word per block pair.
-struct HalfWords {
-  uint32_t p0[4], p1[2], p2[2], p3[4], p4[4];
-};
-
-constexpr uint32_t kMagicBf16 = 0x43004300u;  // bf16 128.0 in both halves
-
-// Kinds of operand a width's MMAs take (decode path):
-//   kOpP0    2-bit value from plane 0 (bits 7..6): width 2, alpha_h = 4^h
-//   kOpNib3  3-bit value from planes 0, 1 (bits 7..5): width 3, alpha = 1
-//   kOpNib4  4-bit value from planes 0, 1, 2 (bits 7..4): width 4 and the high part of 6, 8
-//   kOpP3    2-bit value from plane 3 (bits 3..2): low part of width 6, alpha_h = 4^h
-//   kOpNibLo 4-bit value from planes 3, 4 (bits 3..0): low part of width 8, alpha = 1
-enum { kOpP0 = 0, kOpNib3 = 1, kOpNib4 = 2, kOpP3 = 3, kOpNibLo = 4 };
-
-// alpha of row half h for an operand kind
-__host__ __device__ constexpr int op_alpha(int kind, int h) {
-  return (kind == kOpP0 || kind == kOpP3) ? (h ? 4 : 1) : 1;
-}
-
-// 2-bit plane word x of one block: field f at bits [2f, 2f + 2); register (j, h, kh) has its low
-// half's field at bit 8j + 2h + 4kh and its high half's 16 bits above.
-__device__ __forceinline__ void bf16_from_2bit(uint32_t x, uint32_t (&A)[2][4]) {
-#pragma unroll
-  for (int j = 0; j < 2; ++j)
-#pragma unroll
-    for (int kh = 0; kh < 2; ++kh) {
-      const uint32_t s = x >> (8 * j + 4 * kh);
-      A[j][2 * kh] = and_or(s, 0x00030003u, kMagicBf16);
-      A[j][2 * kh + 1] = and_or(s, 0x000C000Cu, kMagicBf16);
-    }
-}
-// Nibble words C_h (h = 0, 1): nibble n of C_h holds field 2n + h, so register (j, h, kh) has its
-// low half at bit 8j + 4kh of C_h and its high half 16 bits above.
-template <uint32_t kField>
-__device__ __forceinline__ void bf16_from_nibbles(const uint32_t (&C)[2], uint32_t (&A)[2][4]) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int kh = 0; kh < 2; ++kh) A[j][h + 2 * kh] = and_or(C[h] >> (8 * j + 4 * kh), kField, kMagicBf16);
-}
-
-// Operands of block 4*hc + WB (WB in 0..3) of the given kind, from the half-chunk's words.
-template <int KIND, int WB>
-__device__ __forceinline__ void build_bf16(const HalfWords& H, uint32_t (&A)[2][4]) {
-  constexpr int a = WB & 1;  // which block of its 1-bit word
-  if constexpr (KIND == kOpP0) {
-    bf16_from_2bit(H.p0[WB], A);
-  } else if constexpr (KIND == kOpP3) {
-    bf16_from_2bit(H.p3[WB], A);
-  } else if constexpr (KIND == kOpNib3 || KIND == kOpNib4) {
-    uint32_t C[2];
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const uint32_t w0 = H.p0[WB];
-      const uint32_t w1 = H.p1[WB >> 1];
-      if constexpr (KIND == kOpNib3) {
-        // bits 2..1 of a nibble from plane 0, bit 0 from plane 1
-        const uint32_t s0 = (c == 0) ? (w0 << 1) : (w0 >> 1);
-        const uint32_t s1 = w1 >> (2 * a + c);
-        C[c] = bitsel(s0, s1, 0x66666666u);
-      } else {
-        // bits 3..2 from plane 0, bit 1 from plane 1, bit 0 from plane 2
-        const uint32_t w2 = H.p2[WB >> 1];
-        const uint32_t s0 = (c == 0) ? (w0 << 2) : w0;
-        const int sh1 = 1 - 2 * a - c;
-        const uint32_t s1 = sh1 >= 0 ? (w1 << sh1) : (w1 >> (-sh1));
-        const uint32_t s2 = w2 >> (2 * a + c);
-        C[c] = bitsel(bitsel(s0, s1, 0xCCCCCCCCu), s2, 0xEEEEEEEEu);
-      }
-    }
-    bf16_from_nibbles<(KIND == kOpNib3) ? 0x00070007u : 0x000F000Fu>(C, A);
-  } else {
-    // bits 3..2 from plane 3, bits 1..0 from plane 4 (both 2-bit planes, field f at bit 2f)
-    uint32_t C[2];
-#pragma unroll
-    for (int c = 0; c < 2; ++c) C[c] = bitsel(H.p3[WB] << (2 - 2 * c), H.p4[WB] >> (2 * c), 0xCCCCCCCCu);
-    bf16_from_nibbles<0x000F000Fu>(C, A);
-  }
-}
-
 // Operands of block W0 + wb (wb a runtime value in 0..3, resolved by an unrolled switch).
 template <int R, int W0>
 __device__ __forceinline__ void build_slice_operands(const LaneWords& L, int wb, uint32_t (&A)[2][4]) {

@@ -23,8 +23,10 @@
 //
 // fp16 (not bf16) weight tiles: with bf16 y, bf16-rounded weights exceed the 2e-3 relative
 // error budget while fp16 ones stay at the output-rounding level; both formats run at the
-// same tensor-core rate.  x is converted bf16 -> fp16 once per call into the workspace (exact
-// for |x| in the fp16 normal range).
+// same tensor-core rate.  x is converted bf16 -> fp16 once per call into the workspace, each
+// token row first divided by the power of two that keeps its largest value finite in fp16
+// (exact); the epilogue multiplies that token's fp32 results back, so every bf16 input range is
+// served (values more than 2^30 below the row's largest reach fp16's subnormal range).
 //
 // Every mbarrier wait is bounded (about a second of clock); on expiry the kernel records an
 // error code in the workspace header, every role drains, TMEM is freed, and the kernel returns.
@@ -53,23 +55,52 @@ constexpr int kThreads = 32 * (4 + kDeqWarps + kEpiWarps);
 constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
 
 // ---- activation conversion -----------------------------------------------------------------
-__global__ void xprep_prefill_kernel(const uint16_t* __restrict__ x, size_t n, __half* __restrict__ x16) {
+// One block per token row: the row's largest bf16 exponent E gives a power of two 2^e,
+// e = max(0, E - 15), so that every x * 2^-e is a finite fp16 (bf16 values below 2^16 convert
+// exactly; the scaling is exact).  x16 = fp16(x * 2^-e); xscale[m] = 2^e, multiplied back into
+// the token's fp32 results by the epilogue.  Rows whose values all lie below 2^16 keep e = 0.
+constexpr int kXprepThreads = 256;
+__global__ void __launch_bounds__(kXprepThreads) xprep_prefill_kernel(const uint16_t* __restrict__ x, int K,
+                                                                      __half* __restrict__ x16,
+                                                                      float* __restrict__ xscale) {
   pdl_launch_dependents();
   pdl_wait();
-  const size_t nvec = n / 8;
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  for (size_t v = (size_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
-    const uint4 in = reinterpret_cast<const uint4*>(x)[v];
+  const size_t m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(x + m * (size_t)K);
+  uint4* out = reinterpret_cast<uint4*>(x16 + m * (size_t)K);
+  const int nvec = K / 8;
+  // largest exponent field of the row (bf16 bits 14..7)
+  uint32_t emax = 0;
+  for (int v = threadIdx.x; v < nvec; v += kXprepThreads) {
+    const uint4 in = row[v];
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint4 out;
-    uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) emax = max(emax, max((w[i] >> 7) & 0xFFu, (w[i] >> 23) & 0xFFu));
+  }
+  __shared__ uint32_t red[kXprepThreads / 32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = emax;
+  __syncthreads();
+  emax = 0;
+#pragma unroll
+  for (int i = 0; i < kXprepThreads / 32; ++i) emax = max(emax, red[i]);
+  // exponent field 127 + 15 = 142 is the largest that converts without overflow
+  const int e = emax > 142u ? (int)emax - 142 : 0;
+  const float down = __int_as_float((127 - e) << 23);  // 2^-e (e <= 128 for finite inputs)
+  if (threadIdx.x == 0) xscale[m] = __int_as_float((127 + min(e, 127)) << 23);
+  for (int v = threadIdx.x; v < nvec; v += kXprepThreads) {
+    const uint4 in = row[v];
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint4 o4;
+    uint32_t* o = reinterpret_cast<uint32_t*>(&o4);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float a = __uint_as_float(w[i] << 16), b = __uint_as_float(w[i] & 0xFFFF0000u);
+      const float a = __uint_as_float(w[i] << 16) * down, b = __uint_as_float(w[i] & 0xFFFF0000u) * down;
       __half2 h = __floats2half2_rn(a, b);
       o[i] = *reinterpret_cast<uint32_t*>(&h);
     }
-    reinterpret_cast<uint4*>(x16)[v] = out;
+    out[v] = o4;
   }
 }
 
@@ -78,6 +109,7 @@ struct PrefillParams {
   int M, N, K, G, RT;
   const uint16_t* scales;
   const uint8_t* zeros;
+  const float* xscale;  // per token: the power of two its activations were divided by
   void* y;
   int y_mode;
   int* err;
@@ -398,6 +430,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
+        {
+          // tokens whose activations were scaled down get their factor back (warp-uniform test)
+          const int tl = m0 + c * 32 + lane;
+          const float f = tl < P.M ? P.xscale[tl] : 1.f;
+          if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] *= __shfl_sync(0xffffffffu, f, k);
+          }
+        }
         if (P.y_mode == 3) {
           // gated mode: lanes 2i (gate row) and 2i + 1 (up row) share output column n / 2 of
           // y [M, N/2]; the even lane forms tokens 0..15 of the chunk, the odd lane 16..31,
@@ -440,7 +481,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
 }
 
 // ---- host side -----------------------------------------------------------------------------
-size_t prefill_scratch_bytes(int M, int K) { return (((size_t)M * K * 2) + 255) & ~size_t(255); }
+// fp16 copy of x, then one float per token (its scale factor)
+size_t prefill_scratch_bytes(int M, int K) {
+  return ((((size_t)M * K * 2) + 255) & ~size_t(255)) + ((((size_t)M * 4) + 255) & ~size_t(255));
+}
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -504,12 +548,10 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
   uint8_t* ws = (uint8_t*)workspace;
   int* err = (int*)(ws + 4);  // sticky prefill error word in the workspace header
   __half* x16 = (__half*)(ws + workspace_header_bytes());
+  float* xscale = (float*)(ws + workspace_header_bytes() + ((((size_t)M * K * 2) + 255) & ~size_t(255)));
   {
-    const size_t n = (size_t)M * K;
-    int blocks = (int)((n / 8 + 255) / 256);
-    if (blocks > 148 * 8) blocks = 148 * 8;
-    if (blocks < 1) blocks = 1;
-    cudaError_t e = launch_pdl(xprep_prefill_kernel, dim3(blocks), dim3(256), 0, s, (const uint16_t*)x, n, x16);
+    cudaError_t e = launch_pdl(xprep_prefill_kernel, dim3(M), dim3(kXprepThreads), 0, s, (const uint16_t*)x, K, x16,
+                               xscale);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap maps[6];
@@ -537,6 +579,7 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
   P.RT = g.RT;
   P.scales = scales;
   P.zeros = zeros;
+  P.xscale = xscale;
   P.y = y;
   P.y_mode = y_mode;
   P.err = err;

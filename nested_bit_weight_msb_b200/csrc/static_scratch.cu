@@ -16,9 +16,9 @@ using namespace matq;
 
 namespace {
 
-// Capacity of the library-owned scratch.  It holds the workspace header (the status words)
-// and the prefill path's fp16 copy of x while header + M * K * 2 bytes fit (the decode path
-// itself needs only the header).
+// Capacity of the library-owned scratch.  It holds the workspace header (status words and
+// split-row counters) with the decode path's partial-sum slots for any M <= 16, and the
+// prefill path's fp16 copy of x while header + M * K * 2 bytes fit.
 constexpr size_t kStaticScratchBytes = MATQ_NOALLOC_SCRATCH_BYTES;
 
 // One instance per device (the module is loaded into each device's context separately).
@@ -88,9 +88,9 @@ extern "C" int matq_linear_noalloc(const void* x, int M, int K, const void* plan
   st = scratch_for_current_device(&ws);
   if (st) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  // The status words must start at zero.  A call whose device-side wait ran out leaves its
-  // code there, so each call clears the header; the rest of the scratch is written before it
-  // is read.
+  // The header must start at zero.  Every completed call leaves it zero, but one whose
+  // device-side wait ran out does not, so each call clears it; the rest of the scratch is
+  // written before it is read.
   cudaError_t e = cudaMemsetAsync(ws, 0, workspace_header_bytes(), s);
   if (e != cudaSuccess) return record_cuda_error(e);
   st = matq_linear(x, M, K, planes, r_keep, scales, zeros, N, r, group, y, y_mode, ws, kStaticScratchBytes,

@@ -44,6 +44,7 @@ MATQ_OUT_SILU_GATED = 3
 MATQ_SLICE_TRUE_PREFIX = 0
 MATQ_SLICE_TRUNCATE = 1
 MATQ_STATUS_SELFTEST = 0x100
+MATQ_STATUS_XRANGE = 0x200
 
 WIDTHS = (2, 3, 4, 6, 8)
 DECODE_MAX_M = 16

@@ -4,6 +4,9 @@
   in the workspace's status word and lets the kernel return.  matq_selftest_timeout runs that
   wait on a barrier that nothing completes; the host reads the code, the context stays usable,
   and after matq_workspace_init the same workspace serves a correct call again.
+* The decode path's split row groups are combined by the last of their contributors (a ticket
+  from a counter in the workspace header), so a call never waits on another CTA; two calls on
+  unordered streams with their own workspaces both complete with correct results.
 * Canary-padded outputs: nothing is written past the [M, N] (or [M, N/2]) output, for ragged
   rows and token counts on both paths and in every output mode.
 """
@@ -28,7 +31,7 @@ def M():
 
 def test_bounded_wait_times_out_and_is_recoverable(M):
     import torch
-    Mt, N, K, G, r = 1, 4096, 4096, 128, 2
+    Mt, N, K, G, r = 1, 4096, 4096, 128, 2   # 256 items on 148 CTAs: row groups are split
     q, s, z, xb, xv = problem(Mt, N, K, G, seed=21)
     dq, ds, dz, dx = to_device(q, s, z, xb)
     planes = M.pack(dq, r_keep=8)
@@ -45,6 +48,32 @@ def test_bounded_wait_times_out_and_is_recoverable(M):
     assert M.workspace_status(ws) == 0
     rows = np.arange(0, N, 7)
     check_close(y.cpu().numpy()[:, rows], O.linear(xv, q[rows], s[rows], z[rows], r, G), what="after recovery")
+
+
+def test_concurrent_decode_calls_on_unordered_streams(M):
+    """Two decode calls whose row groups are split between CTAs, on two streams with no order
+    between them and their own workspaces: the combine never waits on another CTA, so both
+    finish (whichever CTAs are resident together) with the results of a lone call."""
+    import torch
+    Mt, N, K, G = 1, 8192, 4096, 128
+    q, s, z, xb, xv = problem(Mt, N, K, G, seed=23)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    ref = {r: M.linear(dx, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32).clone() for r in (2, 8)}
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [M.workspace(Mt, K, N, G), M.workspace(Mt, K, N, G)]
+    outs = []
+    for rep in range(4):
+        for i, r in enumerate((2, 8)):
+            with torch.cuda.stream(streams[i]):
+                outs.append((r, M.linear(dx, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32, workspace=wss[i],
+                                         stream=streams[i])))
+    torch.cuda.synchronize()
+    for ws in wss:
+        assert M.workspace_status(ws) == 0
+    for r, y in outs:
+        assert torch.equal(y, ref[r])   # deterministic: the same sums in the same order
 
 
 def _canary(torch, n, dtype):

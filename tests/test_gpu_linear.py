@@ -240,3 +240,81 @@ def test_decode_work_split_paths(M, N, K, Mt):
         assert torch.equal(y1, y2)        # same workspace reused: counters reset, result bitwise stable
         assert M.workspace_status(ws) == 0
         check_close(y1.cpu().numpy()[:, rows], ref, what=f"N={N} K={K} M={Mt} r={r}")
+
+
+def _wide_range_x(rng, Mt, K, lo_exp, hi_exp):
+    """bf16 activations whose magnitudes are log-uniform over [2^lo_exp, 2^hi_exp], random
+    signs, with the extremes present in every row."""
+    e = rng.uniform(lo_exp, hi_exp, (Mt, K))
+    x = np.sign(rng.standard_normal((Mt, K))) * np.exp2(e)
+    x[:, 0] = 2.0 ** lo_exp
+    x[:, 1] = -(2.0 ** hi_exp)
+    return synth.bf16_round(x.astype(np.float32))
+
+
+@pytest.mark.parametrize("r", [2, 8])
+def test_prefill_serves_the_whole_bf16_range(M, r):
+    """Activations from 2^-24 to 2^20 (beyond fp16's 65504): the prefill path divides each token by
+    the power of two that keeps it finite in fp16 and multiplies its results back (exact)."""
+    import torch
+    Mt, N, K, G = 40, 256, 1024, 128
+    q, s, z, _, _ = problem(1, N, K, G, seed=31)
+    rng = np.random.default_rng(r)
+    xb, xv = _wide_range_x(rng, Mt, K, -24, 20)
+    xb[5], xv[5] = synth.bf16_round((rng.standard_normal(K) * 0.5).astype(np.float32))   # an ordinary token too
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    ws = M.workspace(Mt, K, N, G)
+    # The prefill path multiplies fp16 weights s * (q_hat - z) (each within 2^-11 of the exact
+    # value) by fp16 activations x * 2^-e (exact down to 2^-14, then on the subnormal grid of
+    # spacing 2^-24) and accumulates K = 1024 products in fp32 (within 2^-14 of sum |x w|).  With
+    # activations up to 2^20 and random signs, outputs that cancel to near zero sit far below the
+    # products' magnitude, so the bar adds that arithmetic's own bound to the usual one:
+    #   |y - ref| <= 1e-2 (|ref| + 1) + 2^-10 sum_k |x_k w_k| + 2^(e_t - 24) sum_k |w_k|.
+    xf = xv.astype(np.float64)
+    wd = O.dequant(q, s, z, r, G)
+    mag = np.abs(xf) @ np.abs(wd).T
+    e_t = np.maximum(0, np.floor(np.log2(np.max(np.abs(xf), axis=1))) - 15)
+    arith = 2.0 ** -10 * mag + np.exp2(e_t - 24)[:, None] * np.abs(wd).sum(axis=1)[None, :]
+    ref = O.linear(xf, q, s, z, r, G)
+    for mode in (M.MATQ_OUT_F32, M.MATQ_OUT_BF16):
+        y = M.linear(dx, planes, 8, ds, dz, N, r, G, y_mode=mode, workspace=ws)
+        torch.cuda.synchronize()
+        assert M.workspace_status(ws) == 0
+        yh = y.float().cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(yh))
+        err = np.abs(yh - ref)
+        bound = 1e-2 * (np.abs(ref) + 1.0) + arith
+        assert np.all(err <= bound), f"prefill wide x r={r} mode={mode}: worst {np.max(err / bound):.3g}"
+        rel = np.linalg.norm(yh - ref) / np.linalg.norm(ref)
+        assert rel <= 2e-3, f"prefill wide x r={r} mode={mode}: relative Frobenius {rel:.3e}"
+        # the rows whose activations needed no prescale keep the ordinary bar
+        check_close(yh[5:6], ref[5:6], what=f"prefill wide x r={r} mode={mode} ordinary token")
+
+
+@pytest.mark.parametrize("r", [2, 8])
+@pytest.mark.parametrize("Mt", [1, 16])
+def test_decode_input_range(M, r, Mt):
+    """The decode path's fp16 operands: activations from 2^-24 to just below 2^16 match the oracle
+    (values below 2^-14 land on fp16's subnormal grid, far inside the tolerance); one activation
+    of magnitude 2^17 raises MATQ_STATUS_XRANGE in the workspace status."""
+    import torch
+    N, K, G = 4096, 4096, 128
+    q, s, z, _, _ = problem(1, N, K, G, seed=32)
+    rng = np.random.default_rng(10 * r + Mt)
+    xb, xv = _wide_range_x(rng, Mt, K, -24, 15.9)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    ws = M.workspace(Mt, K, N, G)
+    y = M.linear(dx, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32, workspace=ws)
+    torch.cuda.synchronize()
+    assert M.workspace_status(ws) == 0
+    rows = np.sort(np.random.default_rng(7).choice(N, 512, replace=False))
+    check_close(y.cpu().numpy()[:, rows], O.linear(xv.astype(np.float64), q[rows], s[rows], z[rows], r, G),
+                what=f"decode wide x r={r} M={Mt}")
+    big = xb.copy()
+    big[Mt - 1, K // 3] = synth.bf16_round(np.array([2.0 ** 17], dtype=np.float32))[0][0]
+    dbig = torch.from_numpy(big.view(np.int16)).cuda().view(torch.bfloat16)
+    M.linear(dbig, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32, workspace=ws)
+    torch.cuda.synchronize()
+    assert M.workspace_status(ws) & M.MATQ_STATUS_XRANGE

@@ -38,8 +38,8 @@ def test_noalloc_rejects_before_any_launch(M):
     cap = 8 << 20
     assert M.matq_linear_workspace(2048, 4096, 14336, 128) > cap
     assert _call(M, Mt=2048, K=4096, N=14336) == M.MATQ_ESCRATCH
-    assert M.matq_linear_workspace(1024, 4096, 64, 128) > cap
-    assert _call(M, Mt=1024, K=4096) == M.MATQ_ESCRATCH
+    assert M.matq_linear_workspace(992, 4096, 64, 128) > cap
+    assert _call(M, Mt=992, K=4096) == M.MATQ_ESCRATCH
     assert "matq_linear_noalloc" in M.matq_strerror(M.MATQ_ESCRATCH).decode()
 
 
@@ -47,9 +47,9 @@ CASES = [
     # (M, N, K, group, r, y_mode)
     (1, 1000, 1024, 128, 2, 0),       # decode, ragged row tile
     (5, 333, 2560, 64, 3, 1),         # decode, odd M, fp32 out
-    (16, 4096, 4096, 128, 8, 0),      # decode, K split within a cluster
+    (16, 4096, 4096, 128, 8, 0),      # decode, rows split between CTAs
     (64, 1000, 1024, 128, 4, 0),      # prefill path within the fixed scratch
-    (1023, 256, 4096, 128, 6, 1),     # largest M at K = 4096 that fits
+    (991, 256, 4096, 128, 6, 1),      # largest M at K = 4096 that fits
 ]
 
 
