@@ -1263,7 +1263,7 @@ def run_sweep(args):
                     n = len(st["packs"])
                     us = graph_us_per_call(lambda i: matq.linear(xs[name], st["packs"][i % n], 8, st["s"], st["z"], N, r,
                                                                  g, y=y, y_mode=mode, workspace=ws), stream,
-                                           n=min(n, 64))
+                                           n=24)
                     b = linear_bytes(M, N, K, r, group=g, out_cols=cols)
                     fl = 2 * M * N * K
                     gbs, tfs = b / (us * 1e-6) / 1e9, fl / (us * 1e-6) / 1e12

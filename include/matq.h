@@ -202,6 +202,68 @@ int matq_linear(const void* x, int M, int K,
                 void* y, int y_mode,
                 void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- rounded slicing: strict MatQuant and Extra-Precision MatQuant ----------------------- */
+
+/* "Matryoshka Quantization | Summary" §3.2 slices a parent code by rounding instead of
+ * truncating:
+ *     L = floor(q / 2^(8-r) + 1/2)            (0 <= L <= 2^r; ties round up)
+ *     strict MatQuant:          L_c = min(L, 2^r - 1),  W_hat = s * (L_c * 2^(8-r) - z)
+ *     Extra-Precision MatQuant: (same page, §7 Errata) no clamp, W_hat = s * (L * 2^(8-r) - z),
+ *                               2^r + 1 levels; the top one needs an extra bit for the few
+ *                               weights whose codes round up past the last r-bit level.
+ * Rounding needs code bit 7 - r besides the r-bit prefix, so libmatq extracts such a slice
+ * once from a parent pack into
+ *   - a width-r "level pack": MATQ-PL1 planes of width r holding L_c where a code's prefix sits
+ *     (r bits per weight), served by matq_linear_rounded with no centring offset;
+ *   - the overflow list: for each row n, the inputs k (ascending) whose L = 2^r, in CSR form
+ *     (row_ptr [N + 1] int32, cols uint16).  Extra-Precision adds s * 2^(8-r) * x[m, k] to
+ *     y[m, n] for each listed weight (on the prefill path the listed weights' tile values
+ *     become s * (256 - z) instead).
+ * r = 8 rounds nothing: its level pack equals the parent's width-8 planes, its list is empty. */
+
+/* Scratch bytes matq_round_extract needs (4 bytes per (row, 256-input chunk)); 0 if invalid. */
+size_t matq_round_scratch_bytes(int N, int K);
+
+/* Extract the width-r rounded slice of a pack (asynchronous on `stream`).
+ *   planes   parent pack (matq_pack) with r_keep >= the width whose planes hold code bit 7 - r:
+ *            3 for r = 2, 4 for r = 3, 6 for r = 4, 8 for r = 6 and 8 (MATQ_ETRUNC otherwise).
+ *   levels   device buffer of >= matq_packed_bytes(N, K, r) bytes (levels_bytes); written with
+ *            the clamped levels L_c as a width-r pack.
+ *   row_ptr  device [N + 1] int32; written: row n's listed weights are
+ *            cols[row_ptr[n] .. row_ptr[n + 1]); row_ptr[N] is the list's length.
+ *   cols     device uint16 [cols_cap], or NULL.  NULL: only levels and row_ptr are written;
+ *            read row_ptr[N], allocate cols and call again.  Entries at positions >= cols_cap
+ *            are not written.  The kernels that read the list load it in aligned 8-entry
+ *            blocks, so cols must have room for row_ptr[N] rounded up to a multiple of 8.
+ *   scratch  device buffer of >= matq_round_scratch_bytes(N, K) bytes (scratch_bytes).
+ * Shapes: K <= 65536 (uint16 inputs) and N * K < 2^31.  Errors: MATQ_EINVAL_R, MATQ_ETRUNC,
+ * MATQ_EINVAL_SHAPE, MATQ_ENULL, MATQ_EALIGN, MATQ_ESIZE, MATQ_EDEVICE, MATQ_ECUDA. */
+int matq_round_extract(const void* planes, int N, int K, int r_keep, int r,
+                       void* levels, size_t levels_bytes,
+                       int32_t* row_ptr, uint16_t* cols, size_t cols_cap,
+                       void* scratch, size_t scratch_bytes, void* stream);
+
+/* Workspace bytes matq_linear_rounded needs: matq_linear_workspace, plus (M <= 16) room for
+ * an fp32 copy of the dense result [M, N] that the list correction starts from. */
+size_t matq_linear_rounded_workspace(int M, int K, int N, int group);
+
+/* y = x . W_hat^T for a rounded slice (arguments, output modes, workspace rules and input
+ * range as matq_linear, with the level pack in place of the planes and r_keep = r).
+ *   row_ptr, cols  the overflow list from matq_round_extract: Extra-Precision MatQuant.
+ *                  Both NULL: strict MatQuant (the clamped levels alone).  One NULL: MATQ_ENULL.
+ * M <= 16: the decode kernel on the level pack (fp32 result in y, or in the workspace for
+ * bf16 and gated outputs), then one correction kernel that adds the listed weights' terms and
+ * writes y.  M > 16: the prefill kernel, whose dequantising warps overwrite the listed weights'
+ * fp16 tile values; one launch (plus the activation conversion).
+ * Bytes read per call: r * N * K / 8 of levels, the scales and zeros, and 2 bytes per listed
+ * weight (plus row_ptr). */
+int matq_linear_rounded(const void* x, int M, int K,
+                        const void* levels, int r,
+                        const uint16_t* scales, const uint8_t* zeros, int N, int group,
+                        const int32_t* row_ptr, const uint16_t* cols,
+                        void* y, int y_mode,
+                        void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- the sliced linear layer without a caller workspace -------------------------------- */
 
 /* Capacity, in bytes, of the scratch array that libmatq itself holds for matq_linear_noalloc

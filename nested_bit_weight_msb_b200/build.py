@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmatq.so")
-SOURCES = ["api.cu", "pack.cu", "decode.cu", "prefill.cu", "glue.cu", "static_scratch.cu", "choose.cu"]
+SOURCES = ["api.cu", "pack.cu", "decode.cu", "prefill.cu", "rounded.cu", "glue.cu", "static_scratch.cu", "choose.cu"]
 HEADERS = ["common.cuh", "internal.h", "operands.cuh", "sync.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

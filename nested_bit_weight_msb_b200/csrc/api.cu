@@ -190,9 +190,12 @@ int matq_selftest_timeout(void* workspace, size_t ws_bytes, void* stream) {
   return cuda_status(launch_wait_selftest((int*)workspace, MATQ_STATUS_SELFTEST, (cudaStream_t)stream));
 }
 
-int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
-                const uint8_t* zeros, int N, int r, int group, void* y, int y_mode, void* workspace,
-                size_t ws_bytes, void* stream) {
+// The sliced linear with the level offset `delta` added to every stored level before the zero
+// point: delta_r for true-prefix slices (matq_linear), 0 for packs of rounded levels
+// (matq_linear_rounded).
+static int linear_with_delta(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
+                             const uint8_t* zeros, int N, int r, int group, float delta, void* y, int y_mode,
+                             void* workspace, size_t ws_bytes, void* stream) {
   if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
   if (r > r_keep) return MATQ_ETRUNC;
   if (!valid_nk(N, K) || M < 1 || (long long)M * K > (1LL << 40) || (long long)M * N > (1LL << 40))
@@ -211,10 +214,94 @@ int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, con
   const PlaneGeom g = make_geom(N, K);
   cudaError_t e;
   if (M <= kDecodeMaxM)
-    e = launch_decode(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
+    e = launch_decode(x, M, K, planes, g, scales, zeros, r, group, delta, y, y_mode, workspace,
+                      (cudaStream_t)stream);
   else
-    e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, y, y_mode, workspace, (cudaStream_t)stream);
+    e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, delta, nullptr, nullptr, y, y_mode, workspace,
+                       (cudaStream_t)stream);
   return cuda_status(e);
+}
+
+int matq_linear(const void* x, int M, int K, const void* planes, int r_keep, const uint16_t* scales,
+                const uint8_t* zeros, int N, int r, int group, void* y, int y_mode, void* workspace,
+                size_t ws_bytes, void* stream) {
+  const float delta = valid_width(r) ? (float)((1 << (8 - r)) - 1) * 0.5f : 0.f;
+  return linear_with_delta(x, M, K, planes, r_keep, scales, zeros, N, r, group, delta, y, y_mode, workspace,
+                           ws_bytes, stream);
+}
+
+// ---- rounded slicing: strict and Extra-Precision MatQuant -----------------------------------
+
+namespace {
+// The width whose planes hold code bit 7 - r (the bit that rounds the r-bit prefix).
+int rounding_width(int r) { return r == 2 ? 3 : r == 3 ? 4 : r == 4 ? 6 : 8; }
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+}  // namespace
+
+size_t matq_round_scratch_bytes(int N, int K) {
+  if (!valid_nk(N, K)) return 0;
+  return round256((size_t)N * (size_t)(K / kChunk) * sizeof(int));
+}
+
+int matq_round_extract(const void* planes, int N, int K, int r_keep, int r, void* levels, size_t levels_bytes,
+                       int32_t* row_ptr, uint16_t* cols, size_t cols_cap, void* scratch, size_t scratch_bytes,
+                       void* stream) {
+  if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
+  if (r_keep < rounding_width(r)) return MATQ_ETRUNC;
+  if (!valid_nk(N, K) || K > 65536 || (long long)N * K > 0x7FFFFFFFLL) return MATQ_EINVAL_SHAPE;
+  if (!planes || !levels || !row_ptr || !scratch) return MATQ_ENULL;
+  if (!aligned16(planes) || !aligned16(levels) || !aligned16(row_ptr) || !aligned16(scratch) ||
+      (cols && !aligned16(cols)))
+    return MATQ_EALIGN;
+  if (levels_bytes < packed_bytes(N, K, r) || scratch_bytes < matq_round_scratch_bytes(N, K)) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  const PlaneGeom g = make_geom(N, K);
+  return cuda_status(launch_round_extract(planes, g, r, rounding_width(r), levels, (int*)scratch, row_ptr, cols,
+                                          (long long)cols_cap, (cudaStream_t)stream));
+}
+
+size_t matq_linear_rounded_workspace(int M, int K, int N, int group) {
+  const size_t base = matq_linear_workspace(M, K, N, group);
+  if (base == 0 || M > kDecodeMaxM) return base;
+  return round256(base) + round256((size_t)M * (size_t)N * sizeof(float));
+}
+
+int matq_linear_rounded(const void* x, int M, int K, const void* levels, int r, const uint16_t* scales,
+                        const uint8_t* zeros, int N, int group, const int32_t* row_ptr, const uint16_t* cols, void* y,
+                        int y_mode, void* workspace, size_t ws_bytes, void* stream) {
+  if (!valid_width(r)) return MATQ_EINVAL_R;
+  if ((row_ptr == nullptr) != (cols == nullptr)) return MATQ_ENULL;
+  if (!row_ptr)  // strict MatQuant: the clamped levels alone
+    return linear_with_delta(x, M, K, levels, r, scales, zeros, N, r, group, 0.f, y, y_mode, workspace, ws_bytes,
+                             stream);
+  if (!valid_nk(N, K) || M < 1 || K > 65536 || (long long)M * K > (1LL << 40) || (long long)M * N > (1LL << 40))
+    return MATQ_EINVAL_SHAPE;
+  if (M <= kDecodeMaxM && (long long)N > max_decode_rows()) return MATQ_EINVAL_SHAPE;
+  if (group != 64 && group != 128) return MATQ_EINVAL_GROUP;
+  if (y_mode < MATQ_OUT_BF16 || y_mode > MATQ_OUT_SILU_GATED) return MATQ_EDTYPE;
+  if (y_mode == MATQ_OUT_SILU_GATED && (N & 1)) return MATQ_EINVAL_SHAPE;
+  if (!x || !levels || !scales || !zeros || !y || !workspace) return MATQ_ENULL;
+  if (!aligned16(x) || !aligned16(levels) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||
+      !aligned16(workspace) || !aligned16(row_ptr) || !aligned16(cols))
+    return MATQ_EALIGN;
+  if (ws_bytes < matq_linear_rounded_workspace(M, K, N, group)) return MATQ_ESIZE;
+  int st = check_device();
+  if (st) return st;
+  const PlaneGeom g = make_geom(N, K);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (M > kDecodeMaxM)  // the prefill kernel patches the listed weights into its fp16 tiles
+    return cuda_status(launch_prefill(x, M, K, levels, g, scales, zeros, r, group, 0.f, row_ptr, cols, y, y_mode,
+                                      workspace, s));
+  // decode: the dense call, then the correction (in place for fp32 outputs; from an fp32 copy
+  // of the dense result in the workspace for bf16 and gated outputs)
+  const bool in_place = y_mode == MATQ_OUT_F32 || y_mode == MATQ_OUT_F32_ACCUM;
+  float* y32 = in_place ? nullptr
+                        : (float*)((uint8_t*)workspace + round256(matq_linear_workspace(M, K, N, group)));
+  cudaError_t e = launch_decode(x, M, K, levels, g, scales, zeros, r, group, 0.f, in_place ? y : (void*)y32,
+                                in_place ? y_mode : MATQ_OUT_F32, workspace, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_overflow_correct(x, M, K, N, group, r, row_ptr, cols, scales, y32, y, y_mode, s));
 }
 
 int matq_rmsnorm(const float* h, int M, int D, float eps, void* n_out, void* stream) {

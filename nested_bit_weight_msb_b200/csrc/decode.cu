@@ -70,6 +70,7 @@ __host__ __device__ constexpr int rows_per_warp_tiles(int r) { return r <= 4 ? 4
 
 struct DecodeParams {
   int N, K, KC, RT, G, M, y_mode, C, NRG;
+  float delta;  // added to every level before the zero point: delta_r, or 0 for stored levels
   long long I;  // items
   const uint16_t* x;
   const uint16_t* scales;
@@ -173,7 +174,6 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   constexpr int RPW = Lt::RPW, RG = Lt::RG, NG = Lt::NG, KSL = Lt::KSL;
   constexpr int NB = 8 / KSL;                                    // 32-input blocks per slice
   constexpr int kPromoteEvery = (GROUP / 32 < NB) ? GROUP / 32 : NB;  // blocks per scale group part
-  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
   constexpr float kHiScale = (R <= 4) ? 0.0625f : 1.0f;
   // constant A operands: -1024 everywhere (bias removal) and beta per input (token sums)
   constexpr uint32_t kNeg1024 = 0xE400E400u;
@@ -252,7 +252,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
             const float sv = __half2float(*reinterpret_cast<const __half*>(srow + rr * 8 + gl * 2));
             const float zv = (float)zrow[rr * 4 + gl];
             a[h] = sv * amul[h];
-            cz[h] = sv * (kDelta - zv);
+            cz[h] = sv * (P.delta - zv);
           }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
@@ -685,8 +685,8 @@ static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom
 }
 
 cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g, const uint16_t* scales,
-                          const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
-                          cudaStream_t s) {
+                          const uint8_t* zeros, int r, int group, float delta, void* y, int y_mode,
+                          void* workspace, cudaStream_t s) {
   const int NT = (M <= 8) ? 1 : 2;
   uint8_t* ws = (uint8_t*)workspace;
   int sms = sm_count(current_device());
@@ -699,6 +699,7 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
   P.G = K / group;
   P.M = M;
   P.y_mode = y_mode;
+  P.delta = delta;
   P.x = (const uint16_t*)x;
   P.scales = scales;
   P.zeros = zeros;

@@ -17,13 +17,24 @@ size_t decode_workspace_bytes(int M);  // header included
 // Bounded-wait self-test: a kernel whose wait runs out ORs `code` into *err and returns.
 cudaError_t launch_wait_selftest(int* err, int code, cudaStream_t s);
 cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
-                          const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
+                          const uint16_t* scales, const uint8_t* zeros, int r, int group, float delta, void* y,
                           int y_mode, void* workspace, cudaStream_t s);
 
 size_t prefill_scratch_bytes(int M, int K);  // after the header
 cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
-                           const uint16_t* scales, const uint8_t* zeros, int r, int group, void* y,
-                           int y_mode, void* workspace, cudaStream_t s);
+                           const uint16_t* scales, const uint8_t* zeros, int r, int group, float delta,
+                           const int* ovf_row_ptr, const uint16_t* ovf_cols, void* y, int y_mode, void* workspace,
+                           cudaStream_t s);
+
+// Rounded slicing (strict / Extra-Precision MatQuant): the clamped-level pack of width r from
+// a pack holding width r_in's planes, per-(row, chunk) counts in cnt (N * KC ints, replaced by
+// their exclusive prefix sum), row_ptr [N + 1], and (if cols) the listed inputs.
+cudaError_t launch_round_extract(const void* planes, const PlaneGeom& g, int r, int r_in, void* levels, int* cnt,
+                                 int* row_ptr, uint16_t* cols, long long cols_cap, cudaStream_t s);
+// Decode-path correction of the weights listed at level 2^r (see rounded.cu).
+cudaError_t launch_overflow_correct(const void* x, int M, int K, int N, int group, int r, const int* row_ptr,
+                                    const uint16_t* cols, const uint16_t* scales, const float* y32, void* y,
+                                    int y_mode, cudaStream_t s);
 
 cudaError_t launch_rmsnorm(const float* h, int M, int D, float eps, void* out, cudaStream_t s);
 cudaError_t launch_silu_mul(const void* gate, const void* up, int M, int F, void* out, cudaStream_t s);

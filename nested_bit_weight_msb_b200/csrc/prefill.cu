@@ -110,6 +110,11 @@ struct PrefillParams {
   const uint16_t* scales;
   const uint8_t* zeros;
   const float* xscale;  // per token: the power of two its activations were divided by
+  float delta;          // added to every level before the zero point: delta_r, or 0 for stored levels
+  // Extra-Precision MatQuant: rows' lists (CSR, inputs ascending) of the weights whose rounded
+  // level is 2^r, or null.  Their fp16 tile values become s * (256 - z).
+  const int* ovf_row_ptr;
+  const uint16_t* ovf_cols;
   void* y;
   int y_mode;
   int* err;
@@ -242,8 +247,7 @@ __device__ __forceinline__ void load_chunk_meta(ChunkMeta<GROUP>& m, const Prefi
 
 template <int R, int BN, int GROUP, int Q>
 __device__ __forceinline__ void dequant_substage(const LaneWords (&L)[kTilesPerWarp], const ChunkMeta<GROUP>& m,
-                                                 int wq, int lane, uint32_t a_slot) {
-  constexpr float kDelta = (float)((1 << (8 - R)) - 1) * 0.5f;
+                                                 int wq, int lane, uint32_t a_slot, float delta) {
   constexpr int g = (Q * kSubK) / GROUP;  // group of this 64-input slice inside the chunk
 #pragma unroll
   for (int tt = 0; tt < kTilesPerWarp; ++tt) {
@@ -254,7 +258,7 @@ __device__ __forceinline__ void dequant_substage(const LaneWords (&L)[kTilesPerW
       const float sv = __half2float(__ushort_as_half((unsigned short)m.sb[tt][g][h]));
       const float zf = (float)m.zb[tt][g][h];
       s2[h] = __float2half2_rn(sv);
-      dz2[h] = __float2half2_rn(R == 8 ? zf : (kDelta - zf));
+      dz2[h] = __float2half2_rn(R == 8 ? zf : (delta - zf));
     }
     if constexpr (kWarpsPerTile == 1) {
       dequant_block<R, 2 * Q>(L[tt], s2, dz2, a_slot, t, lane);
@@ -266,6 +270,79 @@ __device__ __forceinline__ void dequant_substage(const LaneWords (&L)[kTilesPerW
     }
   }
 }
+
+// Extra-Precision fix-up of the fp16 weight tiles.  Lane l < 16 of a dequantising warp follows
+// the list of row l of the warp's 16-row tile: a 16-entry window of the list (two 16-byte loads
+// from the 8-entry boundary at or below the cursor, none past the row's end), refreshed at each
+// chunk and whenever a slice uses it up, and the fp16 values s * (256 - z) of the chunk's
+// groups.  After the slice's tile is in shared memory the lane overwrites the listed weights of
+// the slice.
+template <int GROUP>
+struct OvfCursor {
+  static constexpr int NG = kChunk / GROUP;
+  int cur = 0, end = 0, base = 0;
+  uint32_t win[8];
+  uint16_t val[NG];
+
+  __device__ __forceinline__ void load_window(const uint16_t* cols) {
+    base = cur & ~7;
+    const uint4 z4 = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+    const uint4 a = base < end ? *reinterpret_cast<const uint4*>(cols + base) : z4;
+    const uint4 b = base + 8 < end ? *reinterpret_cast<const uint4*>(cols + base + 8) : z4;
+    win[0] = a.x; win[1] = a.y; win[2] = a.z; win[3] = a.w;
+    win[4] = b.x; win[5] = b.y; win[6] = b.z; win[7] = b.w;
+  }
+
+  __device__ __forceinline__ void start_tile(const PrefillParams& P, int row) {
+    cur = end = 0;
+    if (row < P.N) {
+      cur = P.ovf_row_ptr[row];
+      end = P.ovf_row_ptr[row + 1];
+    }
+  }
+
+  __device__ __forceinline__ void start_chunk(const PrefillParams& P, int row, int kc) {
+    load_window(P.ovf_cols);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      val[g] = 0;
+      if (row < P.N && cur < end) {
+        const size_t o = (size_t)row * P.G + (size_t)kc * NG + g;
+        const __half s = __ushort_as_half(P.scales[o]);
+        const __half v = __hmul(__float2half_rn(256.f - (float)P.zeros[o]), s);
+        val[g] = __half_as_ushort(v);
+      }
+    }
+  }
+
+  // Overwrite the listed weights with inputs kc*256 + 64q .. +63 in the A slot (row arow of the
+  // 128-row tile, 128-byte swizzled rows of 64 fp16 values).
+  __device__ __forceinline__ void patch(const uint16_t* cols, int kc, int q, uint32_t a_slot, int arow) {
+    const int k0 = kc * kChunk + q * kSubK;
+    for (;;) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int k = (int)((win[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+        if (base + j == cur && cur < end && k < k0 + kSubK) {
+          const int kl = k - k0;
+          const uint32_t addr = a_slot + arow * 128 + ((((kl >> 3) ^ (arow & 7))) << 4) + (kl & 7) * 2;
+          const int gi = (k - kc * kChunk) / GROUP;
+          uint16_t v = val[0];
+#pragma unroll
+          for (int g = 1; g < NG; ++g)
+            if (gi == g) v = val[g];
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+          ++cur;
+        }
+      }
+      if (cur < end && cur >= base + 16) {
+        load_window(cols);  // the slice used the whole window: continue from the cursor
+        continue;
+      }
+      break;
+    }
+  }
+};
 
 template <int R, int BN, int GROUP>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -380,14 +457,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     const int wq = warp - 4;
     bool ok = true;
     int ic = 0, is = 0;  // running chunk and 64-input slice counts
+    static_assert(kTilesPerWarp == 1 && kWarpsPerTile == 1, "the list fix-up assumes one 16-row tile per warp");
+    const bool ovf = P.ovf_row_ptr != nullptr;
+    OvfCursor<GROUP> oc;
     for (int i = 0; i < my_tiles && ok; ++i) {
       const int t = (int)blockIdx.x + i * (int)gridDim.x;
       const int rt0 = (t / MT) * (kBM / kTileRows);
+      const int orow = (rt0 + wq) * kTileRows + lane;  // the row whose list lane (< 16) follows
       ChunkMeta<GROUP> meta;
       load_chunk_meta<GROUP>(meta, P, 0, rt0, wq, lane);
+      if (ovf && lane < 16) oc.start_tile(P, orow);
       for (int kc = 0; kc < KC && ok; ++kc, ++ic) {
         const int rs = ic % kRawStages;
         if (kc > 0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
+        if (ovf && lane < 16) oc.start_chunk(P, orow, kc);
         ok = mbar_wait(&raw_full[rs], (ic / kRawStages) & 1, P.err, 16);
         if (!ok) break;
         const uint8_t* raw = smem + S::kRaw + rs * raw_stage_bytes<R>();
@@ -403,7 +486,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
           ok = mbar_wait(&a_empty[as], ((is / kAStages) & 1) ^ 1, P.err, 32);                  \
           if (ok) {                                                                            \
             const uint32_t a_slot = smem_u32(smem + S::kA + as * kATileBytes);                 \
-            dequant_substage<R, BN, GROUP, Q>(L, meta, wq, lane, a_slot);                      \
+            dequant_substage<R, BN, GROUP, Q>(L, meta, wq, lane, a_slot, P.delta);             \
+            if (ovf) {                                                                         \
+              __syncwarp();                                                                    \
+              if (lane < 16) oc.patch(P.ovf_cols, kc, Q, a_slot, wq * kTileRows + lane);       \
+              __syncwarp();                                                                    \
+            }                                                                                  \
             fence_proxy_async();                                                               \
             mbar_arrive(&a_full[as]);                                                          \
           }                                                                                    \
@@ -543,8 +631,8 @@ static cudaError_t launch_bn(int r, const CUtensorMap (&maps)[6], const PrefillP
 }
 
 cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g, const uint16_t* scales,
-                           const uint8_t* zeros, int r, int group, void* y, int y_mode, void* workspace,
-                           cudaStream_t s) {
+                           const uint8_t* zeros, int r, int group, float delta, const int* ovf_row_ptr,
+                           const uint16_t* ovf_cols, void* y, int y_mode, void* workspace, cudaStream_t s) {
   uint8_t* ws = (uint8_t*)workspace;
   int* err = (int*)(ws + 4);  // sticky prefill error word in the workspace header
   __half* x16 = (__half*)(ws + workspace_header_bytes());
@@ -580,6 +668,9 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
   P.scales = scales;
   P.zeros = zeros;
   P.xscale = xscale;
+  P.delta = delta;
+  P.ovf_row_ptr = ovf_row_ptr;
+  P.ovf_cols = ovf_cols;
   P.y = y;
   P.y_mode = y_mode;
   P.err = err;

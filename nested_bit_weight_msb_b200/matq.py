@@ -66,6 +66,12 @@ _SIGNATURES = {
     "matq_selftest_timeout": (_c_int, [_c_vp, _c_size, _c_vp]),
     "matq_linear": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                              _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
+    "matq_round_scratch_bytes": (_c_size, [_c_int, _c_int]),
+    "matq_round_extract": (_c_int, [_c_vp, _c_int, _c_int, _c_int, _c_int, _c_vp, _c_size, _c_vp, _c_vp, _c_size,
+                                    _c_vp, _c_size, _c_vp]),
+    "matq_linear_rounded_workspace": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "matq_linear_rounded": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_vp,
+                                     _c_vp, _c_vp, _c_int, _c_vp, _c_size, _c_vp]),
     "matq_linear_noalloc": (_c_int, [_c_vp, _c_int, _c_int, _c_vp, _c_int, _c_vp, _c_vp, _c_int, _c_int, _c_int,
                                      _c_vp, _c_int, _c_vp, _c_vp]),
     "matq_rmsnorm": (_c_int, [_c_vp, _c_int, _c_int, _c_float, _c_vp, _c_vp]),
@@ -211,6 +217,62 @@ def linear(x, planes, r_keep: int, scales, zeros, N: int, r: int, group: int, y=
                       _dev(scales, "scales", _dt("float16", "int16"), w), _dev(zeros, "zeros", _dt("uint8"), w),
                       N, r, group, _dev(y, "y", ydt, w), y_mode, _dev(workspace, "workspace", _dt("uint8"), w),
                       workspace.numel(), _stream_ptr(stream)), "matq_linear")
+    return y
+
+
+def round_extract(planes, N: int, K: int, r_keep: int, r: int, stream=None):
+    """The width-r rounded slice of a pack (strict / Extra-Precision MatQuant): returns
+    (levels, row_ptr, cols) -- the clamped-level pack of width r, and the CSR list of the
+    weights whose rounded level is 2^r (cols padded to a multiple of 8 entries).  Reads the
+    list's length back to the host once (a synchronisation of `stream`)."""
+    torch = _torch()
+    w = "round_extract"
+    pp = _dev(planes, "planes", _dt("uint8"), w)
+    dev = planes.device
+    levels = torch.empty(max(matq_packed_bytes(N, K, r), 16), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(N + 1, dtype=torch.int32, device=dev)
+    scratch = torch.empty(max(matq_round_scratch_bytes(N, K), 256), dtype=torch.uint8, device=dev)
+    sp = _stream_ptr(stream)
+    check(matq_round_extract(pp, N, K, r_keep, r, _ptr(levels), levels.numel(), _ptr(row_ptr), None, 0,
+                             _ptr(scratch), scratch.numel(), sp), "matq_round_extract")
+    if stream is not None:
+        stream.synchronize()
+    else:
+        torch.cuda.current_stream(dev).synchronize()
+    nnz = int(row_ptr[N].item())
+    cols = torch.zeros((((nnz + 7) // 8) * 8 + 8,), dtype=torch.int16, device=dev)
+    check(matq_round_extract(pp, N, K, r_keep, r, _ptr(levels), levels.numel(), _ptr(row_ptr), _ptr(cols),
+                             cols.numel(), _ptr(scratch), scratch.numel(), sp), "matq_round_extract")
+    return levels, row_ptr, cols
+
+
+def rounded_workspace(M: int, K: int, N: int, group: int, device="cuda"):
+    torch = _torch()
+    ws = torch.zeros(max(matq_linear_rounded_workspace(M, K, N, group), 256), dtype=torch.uint8, device=device)
+    return ws
+
+
+def linear_rounded(x, levels, r: int, scales, zeros, N: int, group: int, row_ptr=None, cols=None, y=None,
+                   y_mode: int = MATQ_OUT_BF16, workspace=None, stream=None):
+    """y = x . W_hat^T for a rounded slice: Extra-Precision MatQuant with the overflow list
+    (row_ptr, cols from ``round_extract``), strict MatQuant without it."""
+    torch = _torch()
+    M, K = x.shape
+    if y is None:
+        dt = torch.bfloat16 if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else torch.float32
+        ncols = N // 2 if y_mode == MATQ_OUT_SILU_GATED else N
+        y = (torch.zeros if y_mode == MATQ_OUT_F32_ACCUM else torch.empty)((M, ncols), dtype=dt, device=x.device)
+    if workspace is None:
+        workspace = rounded_workspace(M, K, N, group, device=x.device)
+    w = "linear_rounded"
+    ydt = _dt("bfloat16") if y_mode in (MATQ_OUT_BF16, MATQ_OUT_SILU_GATED) else _dt("float32")
+    rp = None if row_ptr is None else _dev(row_ptr, "row_ptr", _dt("int32"), w)
+    cp = None if cols is None else _dev(cols, "cols", _dt("int16", "uint16"), w)
+    check(matq_linear_rounded(_dev(x, "x", _dt("bfloat16"), w), M, K, _dev(levels, "levels", _dt("uint8"), w), r,
+                              _dev(scales, "scales", _dt("float16", "int16"), w), _dev(zeros, "zeros", _dt("uint8"), w),
+                              N, group, rp, cp, _dev(y, "y", ydt, w), y_mode,
+                              _dev(workspace, "workspace", _dt("uint8"), w), workspace.numel(), _stream_ptr(stream)),
+          "matq_linear_rounded")
     return y
 
 

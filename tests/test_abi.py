@@ -178,3 +178,57 @@ def test_choose_codes_rejects(M):
     with pytest.raises(ValueError, match="CUDA tensor"):
         M.choose_codes(torch.zeros((4, 128)), torch.zeros((4, 2), dtype=torch.float16),
                        torch.zeros((4, 2), dtype=torch.uint8), 64)
+
+
+def test_rounded_slicing_queries_and_rejects(M):
+    """Strict / Extra-Precision MatQuant entry points: sizes, and every argument error caught on
+    the host (nothing launches)."""
+    assert M.matq_round_scratch_bytes(28672, 4096) == 28672 * 16 * 4
+    assert M.matq_round_scratch_bytes(17, 512) == 256            # 17 * 2 * 4 bytes, rounded up to 256
+    assert M.matq_round_scratch_bytes(16, 1000) == 0
+    base = M.matq_linear_workspace(16, 4096, 28672, 128)
+    assert M.matq_linear_rounded_workspace(16, 4096, 28672, 128) >= base + 16 * 28672 * 4
+    assert M.matq_linear_rounded_workspace(64, 4096, 28672, 128) == M.matq_linear_workspace(64, 4096, 28672, 128)
+    big = 1 << 30
+
+    def ext(**kw):
+        a = dict(planes=FAKE, N=16, K=1024, r_keep=8, r=2, levels=FAKE, lb=big, row_ptr=FAKE, cols=FAKE,
+                 cap=big, scratch=FAKE, sb=big)
+        a.update(kw)
+        return M.matq_round_extract(a["planes"], a["N"], a["K"], a["r_keep"], a["r"], a["levels"], a["lb"],
+                                    a["row_ptr"], a["cols"], a["cap"], a["scratch"], a["sb"], None)
+
+    assert ext(r=5) == M.MATQ_EINVAL_R
+    # rounding to width r reads code bit 7 - r: widths 3, 4, 6, 8 hold it for r = 2, 3, 4, 6
+    for r, need in ((2, 3), (3, 4), (4, 6), (6, 8)):
+        smaller = {3: 2, 4: 3, 6: 4, 8: 6}[need]
+        assert ext(r=r, r_keep=smaller) == M.MATQ_ETRUNC
+    assert ext(K=1000) == M.MATQ_EINVAL_SHAPE
+    assert ext(K=65536 + 256) == M.MATQ_EINVAL_SHAPE             # inputs are listed as uint16
+    assert ext(N=1 << 20, K=4096) == M.MATQ_EINVAL_SHAPE         # N * K >= 2^31
+    assert ext(row_ptr=None) == M.MATQ_ENULL
+    assert ext(scratch=None) == M.MATQ_ENULL
+    assert ext(cols=FAKE + 2) == M.MATQ_EALIGN
+    assert ext(lb=16 * 1024 * 2 // 8 - 1) == M.MATQ_ESIZE
+    assert ext(sb=4) == M.MATQ_ESIZE
+
+    def lin(**kw):
+        a = dict(x=FAKE, M=1, K=1024, levels=FAKE, r=2, scales=FAKE, zeros=FAKE, N=64, group=128, row_ptr=FAKE,
+                 cols=FAKE, y=FAKE, y_mode=0, ws=FAKE, wsb=big)
+        a.update(kw)
+        return M.matq_linear_rounded(a["x"], a["M"], a["K"], a["levels"], a["r"], a["scales"], a["zeros"], a["N"],
+                                     a["group"], a["row_ptr"], a["cols"], a["y"], a["y_mode"], a["ws"], a["wsb"],
+                                     None)
+
+    assert lin(r=5) == M.MATQ_EINVAL_R
+    assert lin(cols=None) == M.MATQ_ENULL
+    assert lin(row_ptr=None) == M.MATQ_ENULL
+    assert lin(K=1000) == M.MATQ_EINVAL_SHAPE
+    assert lin(group=32) == M.MATQ_EINVAL_GROUP
+    assert lin(y_mode=4) == M.MATQ_EDTYPE
+    assert lin(y_mode=M.MATQ_OUT_SILU_GATED, N=63) == M.MATQ_EINVAL_SHAPE
+    assert lin(row_ptr=FAKE + 4) == M.MATQ_EALIGN
+    assert lin(wsb=M.matq_linear_workspace(1, 1024, 64, 128)) == M.MATQ_ESIZE  # no room for the fp32 copy
+    # without a list (strict MatQuant) the plain linear's checks and workspace apply
+    assert lin(row_ptr=None, cols=None, wsb=16) == M.MATQ_ESIZE
+    assert lin(row_ptr=None, cols=None, x=None) == M.MATQ_ENULL

@@ -30,6 +30,11 @@ def _bf16(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
+def _rne_bf16(a):
+    """fp64 values rounded to the nearest bf16 (ties to even), as fp64."""
+    return synth.bf16_round(np.asarray(a, dtype=np.float32))[1].astype(np.float64)
+
+
 @pytest.mark.parametrize("Mt,D", [(1, 4096), (16, 4096), (33, 1000)])
 def test_rmsnorm(M, Mt, D):
     import torch
@@ -231,3 +236,55 @@ def test_mixnmatch_stack_8b_shapes_sampled(M, Mt):
         check_close(h.cpu().numpy()[:, dcols] - h_before[:, dcols], O.linear(av, q[dcols], s[dcols], z[dcols], r, G),
                     what=f"layer {l} down M={Mt}")
     assert M.workspace_status(ws) == 0
+
+
+def test_stack32_decode_teacher_forced_sampled(M):
+    """The 32-layer Mix'n'Match stack exactly as the stack benchmark serves it (8B FFN shapes,
+    group 128, widths from the seeded {2 x 11, 3 x 10, 4 x 11} permutation, every layer packed
+    keeping only its width's planes, gate+up in one gated call, down accumulating into the fp32
+    residual) at M = 1, checked teacher-forced at every layer: the RMSNorm on all columns, the
+    gated product on 256 sampled columns, the residual update on 256 sampled columns.  The whole
+    pass replayed as the benchmark's CUDA graph must reproduce the layer-by-layer result bit for
+    bit (the kernels sum their partial results in a fixed order)."""
+    import torch
+    import bench
+    weights = bench.host_weights()
+    sb = bench.StackBench(weights, torch.device("cuda", 0), 0)
+    fused = bench.fused_weights(weights)
+    perms = bench.stack_perms()
+    D, F, G = bench.D_MODEL, bench.D_FF, bench.GROUP
+    rng = np.random.default_rng(32)
+    h = sb.h[1]
+    h.copy_(sb.h0[1])
+    for l, lay in enumerate(sb.layers):
+        r = lay["r"]
+        gu, dn = bench.stack_layer_host(fused, perms, l)
+        h_in = h.cpu().numpy().astype(np.float64)
+        sb.layer(lay, 1, h)
+        torch.cuda.synchronize()
+        nv = _bf16(sb.n[1])
+        # both glue outputs are bf16 by definition (bf16 of the fp32 result), so the reference is
+        # the oracle's value rounded to bf16 (unrounded, bf16's own spacing alone is ~2e-3 RMS)
+        check_close(nv, _rne_bf16(O.rmsnorm(h_in, 1e-5)), what=f"layer {l} rmsnorm")
+        cols = np.sort(rng.choice(F, 256, replace=False))
+        g = O.linear(nv, gu[0][2 * cols], gu[1][2 * cols], gu[2][2 * cols], r, G)
+        u = O.linear(nv, gu[0][2 * cols + 1], gu[1][2 * cols + 1], gu[2][2 * cols + 1], r, G)
+        av = _bf16(sb.a[1])
+        check_close(av[:, cols], _rne_bf16(O.gated_product(g, u)), what=f"layer {l} (r={r}) gated gate+up")
+        dcols = np.sort(rng.choice(D, 256, replace=False))
+        check_close(h.cpu().numpy().astype(np.float64)[:, dcols] - h_in[:, dcols],
+                    O.linear(av, dn[0][dcols], dn[1][dcols], dn[2][dcols], r, G), what=f"layer {l} (r={r}) down")
+    assert sb.matq.workspace_status(sb.ws) == 0
+    h_eager = h.clone()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        sb.run(1)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            sb.run(1)
+        h.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+    assert torch.equal(h, h_eager)
+    assert sb.matq.workspace_status(sb.ws) == 0
