@@ -137,7 +137,11 @@ int matq_slice_copy(const void* planes, int N, int K, int r_keep, int r,
 
 /* ---- the sliced linear layer ----------------------------------------------------------- */
 
-/* Workspace bytes matq_linear needs for these sizes (a multiple of 256).
+/* Workspace bytes for matq_linear at these sizes (a multiple of 256): with this much every path
+ * runs in its fastest form.  A prefill call (M > 16) whose matrix leaves most SMs without a
+ * (row block, token tile) splits K and adds partial sums in the workspace; given less room
+ * than that (but at least the header, 262,400 bytes, plus M*K*2 and M*4 bytes, each rounded up
+ * to 256) it runs unsplit.  Decode calls need exactly this size.
  * A workspace starts with a fixed header (device status words and the ticket counters with
  * which the CTAs sharing a split row group elect the one that adds their partial sums; no CTA
  * waits for another).  The header must be zero-filled once before the first call

@@ -81,6 +81,16 @@ int record_cuda_error(cudaError_t e) { return cuda_status(e); }
 int check_sm100_device() { return check_device(); }
 }  // namespace matq
 
+namespace matq {
+size_t linear_workspace_min(int M, int K, int N, int group) {
+  if (M < 1 || N < 1 || K < kChunk || K % kChunk || (group != 64 && group != 128)) return 0;
+  const size_t dec = decode_workspace_bytes(M <= kDecodeMaxM ? M : kDecodeMaxM);
+  if (M <= kDecodeMaxM) return dec;
+  const size_t pre = workspace_header_bytes() + prefill_scratch_min_bytes(M, K);
+  return pre > dec ? pre : dec;
+}
+}  // namespace matq
+
 extern "C" {
 
 int matq_version(void) { return 100; }
@@ -156,9 +166,10 @@ size_t matq_linear_workspace(int M, int K, int N, int group) {
   // sized so that it also serves every smaller M (decode or prefill) with these K, N
   const size_t dec = decode_workspace_bytes(M <= kDecodeMaxM ? M : kDecodeMaxM);
   if (M <= kDecodeMaxM) return dec;
-  const size_t pre = workspace_header_bytes() + prefill_scratch_bytes(M, K);
+  const size_t pre = workspace_header_bytes() + prefill_scratch_bytes(M, K, N);
   return pre > dec ? pre : dec;
 }
+
 
 int matq_workspace_init(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace) return MATQ_ENULL;
@@ -208,7 +219,7 @@ static int linear_with_delta(const void* x, int M, int K, const void* planes, in
   if (!aligned16(x) || !aligned16(planes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y) ||
       !aligned16(workspace))
     return MATQ_EALIGN;
-  if (ws_bytes < matq_linear_workspace(M, K, N, group)) return MATQ_ESIZE;
+  if (ws_bytes < linear_workspace_min(M, K, N, group)) return MATQ_ESIZE;
   int st = check_device();
   if (st) return st;
   const PlaneGeom g = make_geom(N, K);
@@ -218,7 +229,7 @@ static int linear_with_delta(const void* x, int M, int K, const void* planes, in
                       (cudaStream_t)stream);
   else
     e = launch_prefill(x, M, K, planes, g, scales, zeros, r, group, delta, nullptr, nullptr, y, y_mode, workspace,
-                       (cudaStream_t)stream);
+                       ws_bytes, (cudaStream_t)stream);
   return cuda_status(e);
 }
 
@@ -292,7 +303,7 @@ int matq_linear_rounded(const void* x, int M, int K, const void* levels, int r, 
   cudaStream_t s = (cudaStream_t)stream;
   if (M > kDecodeMaxM)  // the prefill kernel patches the listed weights into its fp16 tiles
     return cuda_status(launch_prefill(x, M, K, levels, g, scales, zeros, r, group, 0.f, row_ptr, cols, y, y_mode,
-                                      workspace, s));
+                                      workspace, ws_bytes, s));
   // decode: the dense call, then the correction (in place for fp32 outputs; from an fp32 copy
   // of the dense result in the workspace for bf16 and gated outputs)
   const bool in_place = y_mode == MATQ_OUT_F32 || y_mode == MATQ_OUT_F32_ACCUM;

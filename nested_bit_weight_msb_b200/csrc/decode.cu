@@ -57,11 +57,11 @@ constexpr int kRowSlices = 4;        // warps split an item's row tiles four way
 // register budget of a thread stays at 255, and only two code variants share the I-cache)
 __host__ __device__ constexpr int k_slices(int NT) { return NT > 0 ? 2 : 2; }
 __host__ __device__ constexpr int dec_threads(int NT) { return 32 * kRowSlices * k_slices(NT); }
-// Resident CTAs per SM (CPS): two for M <= 8, r >= 6 on matrices with K <= 4096 (each CTA's 8
-// warps then fit 128 registers a thread, so an SM runs 16 warps and hides more latency; r = 6
-// and 8 carry the most operand-building work per item), otherwise one.  On long-K matrices a
-// row group would be split between too many CTAs; at r <= 4 the gain of the call is lost
-// because two resident CTAs keep the next kernel from starting its prologue early.
+// Resident CTAs per SM (CPS): two for M <= 8 and r in {2, 6, 8} on matrices with K <= 4096
+// (each CTA's 8 warps then fit 128 registers a thread, so an SM runs 16 warps and hides more
+// latency: measured 7% faster at r = 2, the width with the shortest items; r = 6 and 8 carry
+// the most operand-building work per item), otherwise one.  On long-K matrices a row group
+// would be split between too many CTAs; at r = 3 and 4 the call measured slower with two.
 constexpr int kMaxSMs = 160;  // bound on the SMs used, which sizes the partial-sum workspace
 __host__ __device__ constexpr int max_ctas_per_sm(int NT) { return NT == 1 ? 2 : 1; }
 constexpr int kXPitch = kChunk * 2 + 16;  // bytes per activation row in a stage (padded)
@@ -676,7 +676,7 @@ template <int NT, int GROUP, int CPS>
 static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom& g, const DecodeParams& P, int sms,
                                    cudaStream_t s) {
   switch (r) {
-    case 2: return launch_decode_t<2, NT, GROUP, 1>(planes, g, P, sms, s);
+    case 2: return launch_decode_t<2, NT, GROUP, CPS>(planes, g, P, sms, s);
     case 3: return launch_decode_t<3, NT, GROUP, 1>(planes, g, P, sms, s);
     case 4: return launch_decode_t<4, NT, GROUP, 1>(planes, g, P, sms, s);
     case 6: return launch_decode_t<6, NT, GROUP, CPS>(planes, g, P, sms, s);

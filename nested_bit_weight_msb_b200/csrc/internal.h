@@ -20,11 +20,15 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
                           const uint16_t* scales, const uint8_t* zeros, int r, int group, float delta, void* y,
                           int y_mode, void* workspace, cudaStream_t s);
 
-size_t prefill_scratch_bytes(int M, int K);  // after the header
+size_t prefill_scratch_bytes(int M, int K, int N);  // after the header, K-split partial sums included
+size_t prefill_scratch_min_bytes(int M, int K);      // after the header, without them
+int prefill_splits(int M, int K, int N);            // K splits of a prefill call (1: none)
 cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g,
                            const uint16_t* scales, const uint8_t* zeros, int r, int group, float delta,
                            const int* ovf_row_ptr, const uint16_t* ovf_cols, void* y, int y_mode, void* workspace,
-                           cudaStream_t s);
+                           size_t ws_bytes, cudaStream_t s);
+// Smallest workspace a matq_linear call accepts (a prefill call then runs without K splits).
+size_t linear_workspace_min(int M, int K, int N, int group);
 
 // Rounded slicing (strict / Extra-Precision MatQuant): the clamped-level pack of width r from
 // a pack holding width r_in's planes, per-(row, chunk) counts in cnt (N * KC ints, replaced by

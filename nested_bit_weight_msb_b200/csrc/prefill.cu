@@ -107,6 +107,8 @@ __global__ void __launch_bounds__(kXprepThreads) xprep_prefill_kernel(const uint
 // ---- the GEMM kernel -----------------------------------------------------------------------
 struct PrefillParams {
   int M, N, K, G, RT;
+  int S;        // K splits per (row block, token tile); S > 1: fp32 partial sums into `part`
+  float* part;  // [S][M][N] (S > 1), summed and finished by prefill_finish_kernel
   const uint16_t* scales;
   const uint8_t* zeros;
   const float* xscale;  // per token: the power of two its activations were divided by
@@ -293,11 +295,21 @@ struct OvfCursor {
     win[4] = b.x; win[5] = b.y; win[6] = b.z; win[7] = b.w;
   }
 
-  __device__ __forceinline__ void start_tile(const PrefillParams& P, int row) {
+  // the row's list from its first input >= kstart (a K split starts past input 0)
+  __device__ __forceinline__ void start_tile(const PrefillParams& P, int row, int kstart) {
     cur = end = 0;
     if (row < P.N) {
       cur = P.ovf_row_ptr[row];
       end = P.ovf_row_ptr[row + 1];
+      if (kstart > 0) {
+        int lo = cur, hi = end;  // first entry with k >= kstart
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if ((int)P.ovf_cols[mid] < kstart) lo = mid + 1;
+          else hi = mid;
+        }
+        cur = lo;
+      }
     }
   }
 
@@ -366,12 +378,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KC = P.K / kChunk;
-  // Persistent: CTA b takes tiles b, b + grid, ...; tile t = (weight-row block t / MT, token
-  // tile t % MT), token tiles fastest so that the CTAs working on one row block at a time share
-  // its planes through L2.  Two TMEM accumulators: the epilogue of tile i overlaps the MMAs of
-  // tile i + 1.
+  // Persistent: CTA b takes tiles b, b + grid, ...; tile t = (weight-row block, K split, token
+  // tile), token tiles fastest so that the CTAs working on one row block at a time share its
+  // planes through L2.  Two TMEM accumulators: the epilogue of tile i overlaps the MMAs of
+  // tile i + 1.  With S > 1 K splits (small problems: too few tiles for the SMs) each tile
+  // covers chunks [sp*KC/S, (sp+1)*KC/S) and writes fp32 partial sums.
   const int MT = (P.M + BN - 1) / BN;
-  const int tiles = MT * ((P.N + kBM - 1) / kBM);
+  const int tiles = MT * ((P.N + kBM - 1) / kBM) * P.S;
+  // tile t -> (row block, first and end chunk, first token)
+  struct TileCoord { int rb, kc0, kc1, m0, sp; };
+  auto coord = [&](int t) {
+    TileCoord c;
+    const int mt = t % MT, rest = t / MT;
+    c.sp = rest % P.S;
+    c.rb = rest / P.S;
+    c.kc0 = (int)((long long)c.sp * KC / P.S);
+    c.kc1 = (int)((long long)(c.sp + 1) * KC / P.S);
+    c.m0 = mt * BN;
+    return c;
+  };
   const int my_tiles = (tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   constexpr int kNumPlanes = planes_for_width(R);
 
@@ -402,9 +427,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       bool ok = true;
       int ic = 0, ib = 0;  // running chunk (raw ring) and 64-input slice (B ring) counts
       for (int i = 0; i < my_tiles && ok; ++i) {
-        const int t = (int)blockIdx.x + i * (int)gridDim.x;
-        const int m0 = (t % MT) * BN, rt0 = (t / MT) * (kBM / kTileRows);
-        for (int kc = 0; kc < KC && ok; ++kc, ++ic) {
+        const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
+        const int m0 = tc.m0, rt0 = tc.rb * (kBM / kTileRows);
+        for (int kc = tc.kc0; kc < tc.kc1 && ok; ++kc, ++ic) {
           const int rs = ic % kRawStages;
           ok = mbar_wait(&raw_empty[rs], ((ic / kRawStages) & 1) ^ 1, P.err, 1);
           if (!ok) break;
@@ -435,7 +460,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem_d + (uint32_t)(buf * BN);
-        for (int sub = 0; sub < KC * 4 && ok; ++sub, ++is) {
+        const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
+        for (int sub = 0; sub < (tc.kc1 - tc.kc0) * 4 && ok; ++sub, ++is) {
           const int as = is % kAStages, bs = is % kBStages;
           ok = mbar_wait(&a_full[as], (is / kAStages) & 1, P.err, 4) && mbar_wait(&b_full[bs], (is / kBStages) & 1, P.err, 8);
           if (!ok) break;
@@ -461,15 +487,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     const bool ovf = P.ovf_row_ptr != nullptr;
     OvfCursor<GROUP> oc;
     for (int i = 0; i < my_tiles && ok; ++i) {
-      const int t = (int)blockIdx.x + i * (int)gridDim.x;
-      const int rt0 = (t / MT) * (kBM / kTileRows);
+      const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
+      const int rt0 = tc.rb * (kBM / kTileRows);
       const int orow = (rt0 + wq) * kTileRows + lane;  // the row whose list lane (< 16) follows
       ChunkMeta<GROUP> meta;
-      load_chunk_meta<GROUP>(meta, P, 0, rt0, wq, lane);
-      if (ovf && lane < 16) oc.start_tile(P, orow);
-      for (int kc = 0; kc < KC && ok; ++kc, ++ic) {
+      load_chunk_meta<GROUP>(meta, P, tc.kc0, rt0, wq, lane);
+      if (ovf && lane < 16) oc.start_tile(P, orow, tc.kc0 * kChunk);
+      for (int kc = tc.kc0; kc < tc.kc1 && ok; ++kc, ++ic) {
         const int rs = ic % kRawStages;
-        if (kc > 0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
+        if (kc > tc.kc0) load_chunk_meta<GROUP>(meta, P, kc, rt0, wq, lane);
         if (ovf && lane < 16) oc.start_chunk(P, orow, kc);
         ok = mbar_wait(&raw_full[rs], (ic / kRawStages) & 1, P.err, 16);
         if (!ok) break;
@@ -511,8 +537,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       ok = mbar_wait(&acc_full[buf], (i >> 1) & 1, P.err, 64);
       if (!ok) break;
       tc_fence_after();
-      const int t = (int)blockIdx.x + i * (int)gridDim.x;
-      const int m0 = (t % MT) * BN, n = (t / MT) * kBM + 32 * q + lane;
+      const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
+      const int m0 = tc.m0, n = tc.rb * kBM + 32 * q + lane;
       const uint32_t taddr = tmem_d + (uint32_t)(buf * BN) + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -527,7 +553,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
             for (int k = 0; k < 32; ++k) v[k] *= __shfl_sync(0xffffffffu, f, k);
           }
         }
-        if (P.y_mode == 3) {
+        if (P.S > 1) {
+          // K split: this split's fp32 partial sums, finished by prefill_finish_kernel
+          if (n < P.N) {
+            float* part = P.part + (size_t)tc.sp * P.M * P.N;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              const int tok = m0 + c * 32 + k;
+              if (tok < P.M) part[(size_t)tok * P.N + n] = v[k];
+            }
+          }
+        } else if (P.y_mode == 3) {
           // gated mode: lanes 2i (gate row) and 2i + 1 (up row) share output column n / 2 of
           // y [M, N/2]; the even lane forms tokens 0..15 of the chunk, the odd lane 16..31,
           // each taking the value it lacks from its partner
@@ -568,10 +604,61 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   }
 }
 
+// Sum of the S partial results of a K-split call, in split order (deterministic), finished in
+// the call's output mode; one thread per output element (gated: per output column pair).
+__global__ void __launch_bounds__(256) prefill_finish_kernel(const float* __restrict__ part, int S, int M, int N,
+                                                            void* __restrict__ y, int y_mode) {
+  pdl_launch_dependents();
+  pdl_wait();  // the partial sums come from the split kernel
+  const size_t MN = (size_t)M * N;
+  const size_t cols = y_mode == 3 ? (size_t)(N >> 1) : (size_t)N;
+  const size_t total = (size_t)M * cols;
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < total; i += (size_t)gridDim.x * 256) {
+    const size_t m = i / cols, j = i - m * cols;
+    if (y_mode == 3) {
+      const size_t o = m * N + 2 * j;
+      float g = 0.f, u = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        g += part[sp * MN + o];
+        u += part[sp * MN + o + 1];
+      }
+      reinterpret_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * u);
+    } else {
+      float v = 0.f;
+      for (int sp = 0; sp < S; ++sp) v += part[sp * MN + i];
+      if (y_mode == 0) reinterpret_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
+      else if (y_mode == 1) reinterpret_cast<float*>(y)[i] = v;
+      else reinterpret_cast<float*>(y)[i] += v;
+    }
+  }
+}
+
 // ---- host side -----------------------------------------------------------------------------
-// fp16 copy of x, then one float per token (its scale factor)
-size_t prefill_scratch_bytes(int M, int K) {
-  return ((((size_t)M * K * 2) + 255) & ~size_t(255)) + ((((size_t)M * 4) + 255) & ~size_t(255));
+static size_t r256p(size_t b) { return (b + 255) & ~size_t(255); }
+
+static int prefill_bn(int M) { return M <= 64 ? 64 : (M <= 128 ? 128 : 256); }
+
+// K splits of a call: 1 when the (row block, token tile) tiles alone keep at least half the SMs
+// busy; otherwise as many as the SMs allow, each at least two 256-input chunks, at most 8.
+int prefill_splits(int M, int K, int N) {
+  const int sms = sm_count(current_device());
+  const long long tiles = (long long)((M + prefill_bn(M) - 1) / prefill_bn(M)) * ((N + kBM - 1) / kBM);
+  if (2 * tiles >= sms) return 1;
+  long long S = sms / tiles;
+  const int KC = K / kChunk;
+  if (S > KC / 2) S = KC / 2;
+  if (S > 8) S = 8;
+  while (S > 1 && S * M * (long long)N * 4 > (64LL << 20)) --S;  // partial sums: at most 64 MB
+  return S < 2 ? 1 : (int)S;
+}
+
+// fp16 copy of x and one float per token (its scale factor): what every prefill call needs
+size_t prefill_scratch_min_bytes(int M, int K) { return r256p((size_t)M * K * 2) + r256p((size_t)M * 4); }
+
+// ... plus the K-split partial sums, used when the workspace has room for them
+size_t prefill_scratch_bytes(int M, int K, int N) {
+  const int S = prefill_splits(M, K, N);
+  return prefill_scratch_min_bytes(M, K) + (S > 1 ? r256p((size_t)S * M * N * 4) : 0);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -613,10 +700,16 @@ static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P
   }
   // persistent: at most one CTA per SM (the kernel's shared memory allows no second one)
   const int sms = sm_count(dev);
-  const long long tiles = (long long)((P.M + BN - 1) / BN) * ((P.N + kBM - 1) / kBM);
+  const long long tiles = (long long)((P.M + BN - 1) / BN) * ((P.N + kBM - 1) / kBM) * P.S;
   dim3 grid((unsigned)(tiles < sms ? tiles : sms));
-  return launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3], maps[4],
-                    maps[5], P);
+  cudaError_t e = launch_pdl(kern, grid, dim3(kThreads), (size_t)S::kTotal, s, maps[0], maps[1], maps[2], maps[3],
+                             maps[4], maps[5], P);
+  if (e != cudaSuccess || P.S == 1) return e;
+  const long long outs = (long long)P.M * (P.y_mode == 3 ? P.N / 2 : P.N);
+  long long blocks = (outs + 255) / 256;
+  if (blocks > 4 * sms) blocks = 4 * sms;
+  return launch_pdl(prefill_finish_kernel, dim3((unsigned)blocks), dim3(256), 0, s, (const float*)P.part, P.S, P.M,
+                    P.N, P.y, P.y_mode);
 }
 
 template <int BN, int GROUP>
@@ -632,7 +725,8 @@ static cudaError_t launch_bn(int r, const CUtensorMap (&maps)[6], const PrefillP
 
 cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, const PlaneGeom& g, const uint16_t* scales,
                            const uint8_t* zeros, int r, int group, float delta, const int* ovf_row_ptr,
-                           const uint16_t* ovf_cols, void* y, int y_mode, void* workspace, cudaStream_t s) {
+                           const uint16_t* ovf_cols, void* y, int y_mode, void* workspace, size_t ws_bytes,
+                           cudaStream_t s) {
   uint8_t* ws = (uint8_t*)workspace;
   int* err = (int*)(ws + 4);  // sticky prefill error word in the workspace header
   __half* x16 = (__half*)(ws + workspace_header_bytes());
@@ -655,7 +749,7 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
       maps[p] = maps[0];  // unused by this width
     }
   }
-  const int BN = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+  const int BN = prefill_bn(M);
   if (!make_map_2d(&maps[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
                    (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -671,6 +765,8 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
   P.delta = delta;
   P.ovf_row_ptr = ovf_row_ptr;
   P.ovf_cols = ovf_cols;
+  P.S = workspace_header_bytes() + prefill_scratch_bytes(M, K, g.N) <= ws_bytes ? prefill_splits(M, K, g.N) : 1;
+  P.part = (float*)((uint8_t*)xscale + r256p((size_t)M * 4));
   P.y = y;
   P.y_mode = y_mode;
   P.err = err;

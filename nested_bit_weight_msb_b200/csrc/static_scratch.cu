@@ -67,7 +67,7 @@ extern "C" int matq_linear_noalloc(const void* x, int M, int K, const void* plan
   // nothing; then the size check against the fixed capacity.
   if (!valid_width(r) || !valid_width(r_keep)) return MATQ_EINVAL_R;
   if (r > r_keep) return MATQ_ETRUNC;
-  const size_t need = matq_linear_workspace(M, K, N, group);  // 0 for a bad M, K, N or group
+  const size_t need = linear_workspace_min(M, K, N, group);  // 0 for a bad M, K, N or group
   if (N < 1 || M < 1 || K < kChunk || K % kChunk != 0 || (long long)M * K > (1LL << 40) ||
       (long long)M * N > (1LL << 40) || (long long)N * K > (1LL << 40) ||
       (long long)((N + 15) / 16) * (K / kChunk) > (1LL << 31) - 1)

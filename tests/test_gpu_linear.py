@@ -335,3 +335,33 @@ def test_decode_input_range(M, r, Mt):
     M.linear(dbig, planes, 8, ds, dz, N, r, G, y_mode=M.MATQ_OUT_F32, workspace=ws)
     torch.cuda.synchronize()
     assert M.workspace_status(ws) & M.MATQ_STATUS_XRANGE
+
+
+@pytest.mark.parametrize("Mt,N,K,group", [(40, 512, 4096, 128), (130, 264, 2048, 64), (512, 3584, 14336, 64)])
+def test_prefill_k_split(M, Mt, N, K, group):
+    """Small matrices leave most SMs without a (row block, token tile): these three shapes have
+    4, 3 and 56 such tiles for 148 SMs, so the prefill path splits K (8, 8 and 2 ways) and sums
+    the partial results in split order.  Every output mode against the oracle."""
+    import torch
+    q, s, z, xb, xv = problem(Mt, N, K, group, seed=41, outlier_frac=0.01)
+    dq, ds, dz, dx = to_device(q, s, z, xb)
+    planes = M.pack(dq, r_keep=8)
+    rows = np.arange(N) if N <= 512 else np.sort(np.random.default_rng(3).choice(N, 512, replace=False))
+    xf = xv.astype(np.float64)
+    ws = M.workspace(Mt, K, N, group)
+    for r in (2, 8):
+        ref = O.linear(xf, q[rows], s[rows], z[rows], r, group)
+        y32 = M.linear(dx, planes, 8, ds, dz, N, r, group, y_mode=M.MATQ_OUT_F32, workspace=ws)
+        y32 = y32.cpu().numpy().astype(np.float64)
+        check_close(y32[:, rows], ref, what=f"split r={r} M={Mt} N={N}")
+        base = np.random.default_rng(r).standard_normal((Mt, N)).astype(np.float32)
+        ya = torch.from_numpy(base.copy()).cuda()
+        M.linear(dx, planes, 8, ds, dz, N, r, group, y=ya, y_mode=M.MATQ_OUT_F32_ACCUM, workspace=ws)
+        check_close(ya.cpu().numpy()[:, rows] - base[:, rows], ref, what=f"split accum r={r}")
+        yb = M.linear(dx, planes, 8, ds, dz, N, r, group, y_mode=M.MATQ_OUT_BF16, workspace=ws)
+        check_close(yb.float().cpu().numpy()[:, rows], ref, what=f"split bf16 r={r}")
+        ga = M.linear(dx, planes, 8, ds, dz, N, r, group, y_mode=M.MATQ_OUT_SILU_GATED, workspace=ws)
+        gref = O.gated_product(y32[:, 0::2], y32[:, 1::2])
+        err = np.abs(ga.float().cpu().numpy().astype(np.float64) - gref)
+        assert np.all(err <= 2.0 ** -8 * np.abs(gref) + 1e-6), f"split gated r={r}"
+        assert M.workspace_status(ws) == 0

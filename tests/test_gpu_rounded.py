@@ -164,3 +164,17 @@ def test_extra_precision_8b_gate_up_sampled(M, Mt):
     ref = O.gated_product(y32[:, 0::2], y32[:, 1::2])
     err = np.abs(a.float().cpu().numpy().astype(np.float64) - ref)
     assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+
+
+def test_extra_precision_prefill_k_split(M):
+    """A K-split prefill call (N = 264: three 128-row blocks, one token tile, so K = 4096 is
+    split 8 ways) starts each split's list cursor past the split's first input (a binary search
+    in the row's list)."""
+    N, K, G, r, Mt = 264, 4096, 128, 2, 40
+    q, s, z = _problem(N, K, G, seed=33, uniform=True)
+    levels, row_ptr, cols = extract(M, q, r, 3)
+    xb, xv = synth.activations(Mt, K, seed=2)
+    _, ds, dz, dx = to_device(q, s, z, xb)
+    y = M.linear_rounded(dx, levels, r, ds, dz, N, G, row_ptr, cols, y_mode=M.MATQ_OUT_F32)
+    check_close(y.cpu().numpy(), O.linear(xv.astype(np.float64), q, s, z, r, G, mode="extra_precision"),
+                what="extra precision K split")
