@@ -61,6 +61,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode workload only: leave out the prefill sub-record of the default line")
+    ap.add_argument("--no-ep", action="store_true",
+                    help="decode workload only: leave out the Extra-Precision sub-record of the default line")
     ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose", "speedup"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
@@ -480,6 +482,50 @@ def measure(args, spec, fb, stream, world, local, dev):
             "gpu_launches": args.steps * len(fb.calls) * len(FFN_CALLS) * (1 if spec["unit"] == "GB/s" else 2)}
 
 
+EP_WIDTHS = (2, 3, 4)
+
+
+def ep_table(packed, meta, dev, stream, peaks):
+    """Extra-Precision MatQuant ("Matryoshka Quantization | Summary" §7 Errata) per call at M = 1
+    on the 8B FFN matrices: each matrix's rounded slice extracted once from its parent pack (the
+    clamped levels, r bits a weight, plus the list of weights whose rounded level is 2^r), then
+    served by matq_linear_rounded (gate+up with the gated output, down with bf16 output).
+    Algorithmic bytes: the level planes, scales and zeros, 2 bytes per listed weight and the
+    row pointers, x and y.  Each call timed as back-to-back launches over rotating copies."""
+    import torch
+    from nested_bit_weight_msb_b200 import matq, synth
+    out = []
+    for r in EP_WIDTHS:
+        row = {"r": r, "M": 1}
+        for name in ("gate_up", "down"):
+            s, z, N, K = meta[name]
+            levels, row_ptr, cols = matq.round_extract(packed[name][0], N, K, 8, r)
+            nnz = int(row_ptr[-1].item())
+            n_copies = int(min(8, max(2, (256 << 20) // levels.numel() + 1)))
+            lv = [levels] + [levels.clone() for _ in range(n_copies - 1)]
+            lists = [(row_ptr, cols)] + [(row_ptr.clone(), cols.clone()) for _ in range(n_copies - 1)]
+            xb, _ = synth.activations(1, K, seed=0)
+            x = torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16)
+            gated = name == "gate_up"
+            ycols = N // 2 if gated else N
+            y = torch.empty((1, ycols), dtype=torch.bfloat16, device=dev)
+            mode = matq.MATQ_OUT_SILU_GATED if gated else matq.MATQ_OUT_BF16
+            ws = matq.rounded_workspace(1, K, N, GROUP, device=dev)
+            us = graph_us_per_call(lambda i: matq.linear_rounded(x, lv[i % n_copies], r, s, z, N, GROUP,
+                                                                 lists[i % n_copies][0], lists[i % n_copies][1],
+                                                                 y=y, y_mode=mode, workspace=ws), stream)
+            if matq.workspace_status(ws) != 0:
+                raise RuntimeError("device status after the Extra-Precision calls: a call did not complete normally")
+            b = linear_bytes(1, N, K, r, out_cols=ycols) + 2 * nnz + 4 * (N + 1)
+            gbs = b / (us * 1e-6) / 1e9
+            row[name] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 3),
+                         "listed_fraction": round(nnz / (N * K), 5), "bytes": b}
+            del lv, lists, ws
+        out.append(row)
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup()
@@ -511,6 +557,10 @@ def run_ours(args):
         del pfb
         torch.cuda.empty_cache()
 
+    ep = None
+    if args.workload == "ffn8b_decode" and not args.no_ep:
+        ep = ep_table(packed, meta, dev, stream, load_peaks())
+
     if rank == 0:
         peaks = load_peaks()
         line = {
@@ -538,6 +588,10 @@ def run_ours(args):
                 "roofline": pre["roofline"], "e2e": pre["e2e"], "clocks": pre["clocks"], "per_r": pre["per_r"],
                 "gpu_launches": pre["gpu_launches"],
             }
+        if ep is not None:
+            line["extra_precision"] = {"widths": list(EP_WIDTHS), "per_r": ep,
+                                       "note": "rounded slices served from the clamped-level pack plus the list of "
+                                               "weights at level 2^r; the true-prefix calls are in per_r"}
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_oracle_rate(spec, weights)
             if pre is not None:

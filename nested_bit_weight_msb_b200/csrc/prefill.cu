@@ -131,7 +131,7 @@ struct PrefillSmem {
   static constexpr int kB = kA + kAStages * kATileBytes;
   static constexpr int kRaw = kB + kBStages * BN * 128;
   static constexpr int kBar = kRaw + kRawStages * raw_stage_bytes<R>();
-  static constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 4;
+  static constexpr int kNumBars = 2 * kRawStages + 2 * kAStages + 2 * kBStages + 5;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kTotal = kTmemSlot + 16 + 1024;  // + alignment slack
 };
@@ -374,6 +374,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   uint64_t* b_empty = b_full + kBStages;
   uint64_t* acc_full = b_empty + kBStages;   // [2]: accumulator buffer complete (tcgen05.commit)
   uint64_t* acc_empty = acc_full + 2;        // [2]: accumulator buffer drained by the epilogue
+  uint64_t* drain = acc_empty + 2;           // error path: completion of every MMA issued
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -405,6 +406,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     for (int i = 0; i < kAStages; ++i) { mbar_init(&a_full[i], 32 * kDeqWarps); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < kBStages; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], kEpiWarps); }
+    mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -426,6 +428,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
       const CUtensorMap* maps[5] = {&tm_p0, &tm_p1, &tm_p2, &tm_p3, &tm_p4};
       bool ok = true;
       int ic = 0, ib = 0;  // running chunk (raw ring) and 64-input slice (B ring) counts
+      int ic_sent = 0, ib_sent = 0;  // loads issued (the error path waits for the last of them)
       for (int i = 0; i < my_tiles && ok; ++i) {
         const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
         const int m0 = tc.m0, rt0 = tc.rb * (kBM / kTileRows);
@@ -438,14 +441,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
 #pragma unroll
           for (int p = 0; p < kNumPlanes; ++p)
             tma_load_2d(raw + raw_plane_off(p), maps[p], kc * plane_bits(p) * 64, rt0, &raw_full[rs]);
+          ic_sent = ic + 1;
           for (int q = 0; q < 4; ++q, ++ib) {
             const int bs = ib % kBStages;
             ok = mbar_wait(&b_empty[bs], ((ib / kBStages) & 1) ^ 1, P.err, 2);
             if (!ok) break;
             mbar_expect_tx(&b_full[bs], BN * 128);
             tma_load_2d(smem + S::kB + bs * BN * 128, &tm_x, kc * kChunk + q * kSubK, m0, &b_full[bs]);
+            ib_sent = ib + 1;
           }
         }
+      }
+      if (!ok) {
+        // error path: no copy may still be landing in shared memory when the CTA exits; every
+        // load before the last ring's worth was consumed before its slot was reused
+        for (int c = ic_sent > kRawStages ? ic_sent - kRawStages : 0; c < ic_sent; ++c)
+          mbar_wait(&raw_full[c % kRawStages], (c / kRawStages) & 1, P.err, 1);
+        for (int c = ib_sent > kBStages ? ib_sent - kBStages : 0; c < ib_sent; ++c)
+          mbar_wait(&b_full[c % kBStages], (c / kBStages) & 1, P.err, 2);
       }
     }
   } else if (warp == 1) {
@@ -476,6 +489,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
           tc_commit(&b_empty[bs]);
         }
         if (ok) tc_commit(&acc_full[buf]);
+      }
+      if (!ok) {
+        // error path: wait (bounded) until every MMA issued so far has completed, before the
+        // accumulators are deallocated
+        tc_commit(drain);
+        mbar_wait(drain, 0, P.err, 4);
       }
     }
   } else if (warp >= 4 && warp < 4 + kDeqWarps) {
