@@ -63,7 +63,7 @@ def parse():
                     help="decode workload only: leave out the prefill sub-record of the default line")
     ap.add_argument("--no-ep", action="store_true",
                     help="decode workload only: leave out the Extra-Precision sub-record of the default line")
-    ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose", "speedup"], default=None,
+    ap.add_argument("--case", choices=["decode", "prefill", "pack", "choose", "speedup", "ep"], default=None,
                     help="profiling aid: run a few single sliced-linear calls on the 8B gate matrix and exit")
     ap.add_argument("--r", type=int, default=2)
     ap.add_argument("--m", type=int, default=1)
@@ -1401,7 +1401,8 @@ def run_case(args):
     """A few single calls of the gate+up projection (28672 x 4096 row-interleaved, group 128,
     gated-product epilogue, as in the workloads) at width r and batch m, rotating through
     device copies of the pack (> L2); used for ncu captures.
-    `--case pack` times the one-time pack instead."""
+    `--case pack` times the one-time pack instead; `--case ep` makes the same calls on the
+    Extra-Precision slice (clamped-level pack plus overflow list) of width r."""
     if args.case == "choose":
         return run_choose_case(args)
     if args.case == "speedup":
@@ -1423,7 +1424,13 @@ def run_case(args):
     gated = True
     y = torch.empty((args.m, N // 2 if gated else N), dtype=torch.bfloat16, device="cuda")
     mode = matq.MATQ_OUT_SILU_GATED if gated else matq.MATQ_OUT_BF16
-    for i in range(args.calls):
+    if args.case == "ep":
+        slices = [matq.round_extract(p, N, D_MODEL, 8, args.r) for p in packs]
+        ws = matq.rounded_workspace(args.m, D_MODEL, N, GROUP)
+        for i in range(args.calls):
+            lv, rp, cl = slices[i % len(slices)]
+            matq.linear_rounded(dx, lv, args.r, ds, dz, N, GROUP, rp, cl, y=y, y_mode=mode, workspace=ws)
+    for i in range(args.calls if args.case != "ep" else 0):
         matq.linear(dx, packs[i % len(packs)], 8, ds, dz, N, args.r, GROUP, y=y, y_mode=mode, workspace=ws)
     torch.cuda.synchronize()
     assert matq.workspace_status(ws) == 0

@@ -60,6 +60,22 @@ constexpr int kATileBytes = kBM * kSubK * 2;  // 16 KB
 // exactly; the scaling is exact).  x16 = fp16(x * 2^-e); xscale[m] = 2^e, multiplied back into
 // the token's fp32 results by the epilogue.  Rows whose values all lie below 2^16 keep e = 0.
 constexpr int kXprepThreads = 256;
+constexpr int kXprepHeld = 8;  // 16-byte vectors a thread keeps in registers (rows of K <= 16384)
+__device__ __forceinline__ uint32_t bf16x2_emax(uint32_t w) {
+  return max((w >> 7) & 0xFFu, (w >> 23) & 0xFFu);
+}
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 in, float down) {
+  const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  uint4 o4;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&o4);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = __uint_as_float(w[i] << 16) * down, b = __uint_as_float(w[i] & 0xFFFF0000u) * down;
+    __half2 h = __floats2half2_rn(a, b);
+    o[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  return o4;
+}
 __global__ void __launch_bounds__(kXprepThreads) xprep_prefill_kernel(const uint16_t* __restrict__ x, int K,
                                                                       __half* __restrict__ x16,
                                                                       float* __restrict__ xscale) {
@@ -69,13 +85,24 @@ __global__ void __launch_bounds__(kXprepThreads) xprep_prefill_kernel(const uint
   const uint4* row = reinterpret_cast<const uint4*>(x + m * (size_t)K);
   uint4* out = reinterpret_cast<uint4*>(x16 + m * (size_t)K);
   const int nvec = K / 8;
+  const bool held = nvec <= kXprepHeld * kXprepThreads;  // the row is read once, kept in registers
+  uint4 v[kXprepHeld];
   // largest exponent field of the row (bf16 bits 14..7)
   uint32_t emax = 0;
-  for (int v = threadIdx.x; v < nvec; v += kXprepThreads) {
-    const uint4 in = row[v];
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+  if (held) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) emax = max(emax, max((w[i] >> 7) & 0xFFu, (w[i] >> 23) & 0xFFu));
+    for (int u = 0; u < kXprepHeld; ++u) {
+      const int i = threadIdx.x + u * kXprepThreads;
+      v[u] = i < nvec ? row[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kXprepHeld; ++u)
+      emax = max(emax, max(max(bf16x2_emax(v[u].x), bf16x2_emax(v[u].y)), max(bf16x2_emax(v[u].z), bf16x2_emax(v[u].w))));
+  } else {
+    for (int i = threadIdx.x; i < nvec; i += kXprepThreads) {
+      const uint4 in = row[i];
+      emax = max(emax, max(max(bf16x2_emax(in.x), bf16x2_emax(in.y)), max(bf16x2_emax(in.z), bf16x2_emax(in.w))));
+    }
   }
   __shared__ uint32_t red[kXprepThreads / 32];
 #pragma unroll
@@ -89,18 +116,14 @@ __global__ void __launch_bounds__(kXprepThreads) xprep_prefill_kernel(const uint
   const int e = emax > 142u ? (int)emax - 142 : 0;
   const float down = __int_as_float((127 - e) << 23);  // 2^-e (e <= 128 for finite inputs)
   if (threadIdx.x == 0) xscale[m] = __int_as_float((127 + min(e, 127)) << 23);
-  for (int v = threadIdx.x; v < nvec; v += kXprepThreads) {
-    const uint4 in = row[v];
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint4 o4;
-    uint32_t* o = reinterpret_cast<uint32_t*>(&o4);
+  if (held) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a = __uint_as_float(w[i] << 16) * down, b = __uint_as_float(w[i] & 0xFFFF0000u) * down;
-      __half2 h = __floats2half2_rn(a, b);
-      o[i] = *reinterpret_cast<uint32_t*>(&h);
+    for (int u = 0; u < kXprepHeld; ++u) {
+      const int i = threadIdx.x + u * kXprepThreads;
+      if (i < nvec) out[i] = bf16x8_to_f16x8(v[u], down);
     }
-    out[v] = o4;
+  } else {
+    for (int i = threadIdx.x; i < nvec; i += kXprepThreads) out[i] = bf16x8_to_f16x8(row[i], down);
   }
 }
 
@@ -273,7 +296,8 @@ __device__ __forceinline__ void dequant_substage(const LaneWords (&L)[kTilesPerW
   }
 }
 
-// Extra-Precision fix-up of the fp16 weight tiles.  Lane l < 16 of a dequantising warp follows
+// Extra-Precision fix-up of the fp16 weight tiles (compiled only into the kernels for calls with
+// a list, so the dequantising loop of every other call carries none of it).  Lane l < 16 of a dequantising warp follows
 // the list of row l of the warp's 16-row tile: a 16-entry window of the list (two 16-byte loads
 // from the 8-entry boundary at or below the cursor, none past the row's end), refreshed at each
 // chunk and whenever a slice uses it up, and the fp16 values s * (256 - z) of the chunk's
@@ -356,7 +380,7 @@ struct OvfCursor {
   }
 };
 
-template <int R, int BN, int GROUP>
+template <int R, int BN, int GROUP, bool EP, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant__ CUtensorMap tm_p1,
                const __grid_constant__ CUtensorMap tm_p2, const __grid_constant__ CUtensorMap tm_p3,
@@ -385,16 +409,24 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
   // tile i + 1.  With S > 1 K splits (small problems: too few tiles for the SMs) each tile
   // covers chunks [sp*KC/S, (sp+1)*KC/S) and writes fp32 partial sums.
   const int MT = (P.M + BN - 1) / BN;
-  const int tiles = MT * ((P.N + kBM - 1) / kBM) * P.S;
+  const int NS = SPLIT ? P.S : 1;  // K splits (compiled in only where a call splits)
+  const int tiles = MT * ((P.N + kBM - 1) / kBM) * NS;
   // tile t -> (row block, first and end chunk, first token)
   struct TileCoord { int rb, kc0, kc1, m0, sp; };
   auto coord = [&](int t) {
     TileCoord c;
     const int mt = t % MT, rest = t / MT;
-    c.sp = rest % P.S;
-    c.rb = rest / P.S;
-    c.kc0 = (int)((long long)c.sp * KC / P.S);
-    c.kc1 = (int)((long long)(c.sp + 1) * KC / P.S);
+    if constexpr (SPLIT) {
+      c.sp = rest % NS;
+      c.rb = rest / NS;
+      c.kc0 = (int)((long long)c.sp * KC / NS);
+      c.kc1 = (int)((long long)(c.sp + 1) * KC / NS);
+    } else {
+      c.sp = 0;
+      c.rb = rest;
+      c.kc0 = 0;
+      c.kc1 = KC;
+    }
     c.m0 = mt * BN;
     return c;
   };
@@ -503,7 +535,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
     bool ok = true;
     int ic = 0, is = 0;  // running chunk and 64-input slice counts
     static_assert(kTilesPerWarp == 1 && kWarpsPerTile == 1, "the list fix-up assumes one 16-row tile per warp");
-    const bool ovf = P.ovf_row_ptr != nullptr;
+    constexpr bool ovf = EP;  // Extra-Precision list given (P.ovf_row_ptr non-null)
     OvfCursor<GROUP> oc;
     for (int i = 0; i < my_tiles && ok; ++i) {
       const TileCoord tc = coord((int)blockIdx.x + i * (int)gridDim.x);
@@ -572,7 +604,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_p0, const __grid_constant_
             for (int k = 0; k < 32; ++k) v[k] *= __shfl_sync(0xffffffffu, f, k);
           }
         }
-        if (P.S > 1) {
+        if (SPLIT) {
           // K split: this split's fp32 partial sums, finished by prefill_finish_kernel
           if (n < P.N) {
             float* part = P.part + (size_t)tc.sp * P.M * P.N;
@@ -704,10 +736,10 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int R, int BN, int GROUP>
+template <int R, int BN, int GROUP, bool EP, bool SPLIT>
 static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
   using S = PrefillSmem<R, BN>;
-  auto kern = prefill_kernel<R, BN, GROUP>;
+  auto kern = prefill_kernel<R, BN, GROUP, EP, SPLIT>;
   // the shared-memory attribute is set once per device for this kernel
   static std::atomic<unsigned long long> attr_set{0};
   const int dev = current_device();
@@ -731,14 +763,28 @@ static cudaError_t launch_t(const CUtensorMap (&maps)[6], const PrefillParams& P
                     P.N, P.y, P.y_mode);
 }
 
+template <int BN, int GROUP, bool SPLIT>
+static cudaError_t launch_bn_split(int r, const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
+  switch (r) {
+    case 2: return launch_t<2, BN, GROUP, false, SPLIT>(maps, P, s);
+    case 3: return launch_t<3, BN, GROUP, false, SPLIT>(maps, P, s);
+    case 4: return launch_t<4, BN, GROUP, false, SPLIT>(maps, P, s);
+    case 6: return launch_t<6, BN, GROUP, false, SPLIT>(maps, P, s);
+    default: return launch_t<8, BN, GROUP, false, SPLIT>(maps, P, s);
+  }
+}
+
+// Kernel variants: true-prefix calls unsplit or K-split; Extra-Precision calls (the list
+// fix-up compiled in, r < 8 only: width 8 rounds nothing) unsplit.
 template <int BN, int GROUP>
 static cudaError_t launch_bn(int r, const CUtensorMap (&maps)[6], const PrefillParams& P, cudaStream_t s) {
+  if (P.ovf_row_ptr == nullptr || r == 8)
+    return P.S > 1 ? launch_bn_split<BN, GROUP, true>(r, maps, P, s) : launch_bn_split<BN, GROUP, false>(r, maps, P, s);
   switch (r) {
-    case 2: return launch_t<2, BN, GROUP>(maps, P, s);
-    case 3: return launch_t<3, BN, GROUP>(maps, P, s);
-    case 4: return launch_t<4, BN, GROUP>(maps, P, s);
-    case 6: return launch_t<6, BN, GROUP>(maps, P, s);
-    default: return launch_t<8, BN, GROUP>(maps, P, s);
+    case 2: return launch_t<2, BN, GROUP, true, false>(maps, P, s);
+    case 3: return launch_t<3, BN, GROUP, true, false>(maps, P, s);
+    case 4: return launch_t<4, BN, GROUP, true, false>(maps, P, s);
+    default: return launch_t<6, BN, GROUP, true, false>(maps, P, s);
   }
 }
 
@@ -784,7 +830,10 @@ cudaError_t launch_prefill(const void* x, int M, int K, const void* planes, cons
   P.delta = delta;
   P.ovf_row_ptr = ovf_row_ptr;
   P.ovf_cols = ovf_cols;
-  P.S = workspace_header_bytes() + prefill_scratch_bytes(M, K, g.N) <= ws_bytes ? prefill_splits(M, K, g.N) : 1;
+  // K splits: when the workspace has room for the partial sums; Extra-Precision calls do not split
+  P.S = (ovf_row_ptr == nullptr && workspace_header_bytes() + prefill_scratch_bytes(M, K, g.N) <= ws_bytes)
+            ? prefill_splits(M, K, g.N)
+            : 1;
   P.part = (float*)((uint8_t*)xscale + r256p((size_t)M * 4));
   P.y = y;
   P.y_mode = y_mode;
