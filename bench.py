@@ -621,10 +621,10 @@ _KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
 NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
-    "decode": {"sha256": "0532170b3041f920007ae78a117291f110bc4db70afbe0a4056be508aefd1756", "launch": "gate_up gated 28672x4096 r=2 M=1",
-               "bytes": 32_189_952 + 0},
-    "prefill": {"sha256": "db3339a9714ea591b690c3e5b188aba3558a03759e92efc1d78c9ba8c6cbd491", "launch": "gate_up gated 28672x4096 r=4 M=2048",
-                "bytes": 78_311_168 + 31_010_048},
+    "decode": {"sha256": "f7e9ecb7727bd439ab668b1315624a109a3949ad356731e45413f3525843986f", "launch": "gate_up gated 28672x4096 r=2 M=1",
+               "bytes": 32_188_672 + 0},
+    "prefill": {"sha256": "58199cae351b8d6212fb20b4465a2ca14b7fd9a967156d6ed4862827fef8cb53", "launch": "gate_up gated 28672x4096 r=4 M=2048",
+                "bytes": 78_321_664 + 30_037_760},
 }
 
 
