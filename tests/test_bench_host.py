@@ -83,3 +83,61 @@ def test_choose_case_cpu_baseline_is_bounded_and_well_formed():
     assert rec["kind"] == "oracle" and rec["unit"] == "Gweights/s"
     assert rec["value"] > 0 and rec["cores"] >= 1
     assert "1 rows" in rec["sample"] and "pass" in rec["sample"]
+
+
+def test_stack_permutations_keep_gate_up_pairs_and_are_distinct():
+    """The stack's layers are row-permuted copies of the seeded 8B layer: gate+up rows move in
+    pairs (row 2i gate, 2i + 1 up of the same output channel), down rows singly; every layer's
+    permutation is a bijection and layers differ."""
+    perms = bench.stack_perms(layers=3)
+    for pp, pd in perms:
+        assert sorted(pp.tolist()) == list(range(bench.D_FF))
+        assert sorted(pd.tolist()) == list(range(bench.D_MODEL))
+        rows = bench.stack_rows(pp)
+        assert np.array_equal(rows[0::2], 2 * pp) and np.array_equal(rows[1::2], 2 * pp + 1)
+    assert not np.array_equal(perms[0][0], perms[1][0])
+    assert np.array_equal(bench.stack_perms(layers=3)[2][1], perms[2][1])   # seeded
+
+
+def test_stack_layer_host_moves_codes_scales_and_zeros_together():
+    rng = np.random.default_rng(1)
+    F, D, G = bench.D_FF, bench.D_MODEL, bench.GROUP
+    fused = {"gate_up": (np.arange(2 * F, dtype=np.int64)[:, None] * np.ones((1, 2)), np.arange(2 * F)[:, None],
+                         -np.arange(2 * F)[:, None]),
+             "down": (np.arange(D)[:, None] * np.ones((1, 2)), np.arange(D)[:, None], -np.arange(D)[:, None])}
+    perms = bench.stack_perms(layers=2)
+    gu, dn = bench.stack_layer_host(fused, perms, 1)
+    idx = bench.stack_rows(perms[1][0])
+    assert np.array_equal(gu[0][:, 0], idx) and np.array_equal(gu[1][:, 0], idx) and np.array_equal(gu[2][:, 0], -idx)
+    assert np.array_equal(dn[0][:, 0], perms[1][1]) and np.array_equal(dn[2][:, 0], -perms[1][1])
+    del rng, G
+
+
+def test_stack_units_count_each_layer_once():
+    """One pass: per layer the gated gate+up call (bf16 out, N/2 columns) and the down call into
+    the fp32 residual (read and written); flops 2 M (2F D + D F) per layer."""
+    widths = [2, 3, 4]
+    b, f = bench.stack_units(1, widths)
+    D, F, G = bench.D_MODEL, bench.D_FF, bench.GROUP
+    want = 0
+    for r in widths:
+        want += 2 * F * D * r // 8 + 2 * F * (D // G) * 3 + D * 2 + F * 2
+        want += D * F * r // 8 + D * (F // G) * 3 + F * 2 + D * 8
+    assert b == want
+    assert f == len(widths) * 2 * (2 * F * D + D * F)
+
+
+def test_sweep_shapes_and_configs():
+    sw = bench.SWEEPS["ffn9b_sweep"]
+    assert sw["group"] == 64 and sw["batches"] == (1, 8, 32, 128, 512, 2048) and tuple(sw["widths"]) == (2, 3, 4, 6, 8)
+    one = bench.SWEEPS["linear1024"]
+    assert (one["n"], one["k"], one["group"], one["batches"]) == (1024, 1024, 128, (1,))
+    import argparse
+    cfg = bench.sweep_config(argparse.Namespace(workload="ffn9b_sweep"), sw, {"gate_up": [28672, 3584]}, 1)
+    assert cfg["workload"] == "ffn9b_sweep" and cfg["group"] == 64 and cfg["batches"][-1] == 2048
+
+
+def test_linear_bytes_counts_exactly_r_bits_a_weight():
+    for r in (2, 3, 4, 6, 8):
+        b = bench.linear_bytes(1, 4096, 14336, r)
+        assert b == 4096 * 14336 * r // 8 + 4096 * (14336 // 128) * 3 + 14336 * 2 + 4096 * 2
