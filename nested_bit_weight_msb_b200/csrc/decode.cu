@@ -166,8 +166,10 @@ __device__ __forceinline__ long long item_owner(long long u, long long I, long l
 }
 
 // Work of one warp: RPW row tiles (row slice rs) x input slice KS of every item.
+// Returns the number of ring refills this warp issued (warp 0's count is the TMA requests
+// beyond the prologue).
 template <int R, int NT, int GROUP, int CPS, int KS, typename Refill>
-__device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem, uint64_t* full, uint64_t* empty,
+__device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem, uint64_t* full, uint64_t* empty,
                                             float* red, long long c, long long ib, long long ie, int rs, int lane,
                                             Refill&& refill) {
   using Lt = DecodeLayout<R, NT, GROUP, CPS>;
@@ -207,6 +209,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   // (row group, chunk) of the current item, advanced item by item (no division in the loop)
   const int rg_first = (int)(ib / P.KC);
   int rg = rg_first, kc = (int)(ib - (long long)rg_first * P.KC);
+  int refills = 0;
   for (int n = 0; n < nitems; ++n) {
     const int s = n % Lt::kStages;
     if (ok) ok = mbar_wait(&full[s], (n / Lt::kStages) & 1, P.err, 2);
@@ -303,6 +306,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
           ++rg2;
         }
         refill(n + Lt::kStages, rg2, kc2);
+        ++refills;
       }
     }
 
@@ -464,6 +468,7 @@ __device__ __forceinline__ void decode_warp(const DecodeParams& P, uint8_t* smem
   // the call's outputs are undefined and the status word says so
   const uint32_t big = max(xmax >> 16, xmax & 0xFFFFu);
   if (__any_sync(0xffffffffu, big >= 0x4780u) && lane == 0) atomicOr(P.err, MATQ_STATUS_XRANGE);
+  return refills;
 }
 
 template <int R, int NT, int GROUP, int CPS>
@@ -577,8 +582,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
 
   const int rs = warp & 3, ks = warp >> 2;
   static_assert(Lt::KSL == 2, "two input slices per item");
-  if (ks == 0) decode_warp<R, NT, GROUP, CPS, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
-  else decode_warp<R, NT, GROUP, CPS, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+  const int refills = ks == 0 ? decode_warp<R, NT, GROUP, CPS, 0>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill)
+                              : decode_warp<R, NT, GROUP, CPS, 1>(P, smem, full, empty, red, c, ib, ie, rs, lane, refill);
+  // No copy may still be landing in shared memory when the CTA exits (after a bounded wait
+  // gave up, items requested may not have been consumed): each thread's cp.async copies, then
+  // thread 0 waits (bounded) for the ring's last requested items.  Every phase has completed on
+  // the normal path, so these waits return at once.
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int req = pre + refills;
+    for (int i = req > Lt::kStages ? req - Lt::kStages : 0; i < req; ++i)
+      mbar_wait(&full[i % Lt::kStages], (i / Lt::kStages) & 1, P.err, 2);
+  }
 }
 
 // Failure-detection self-test: one warp waits, with the bounded wait every kernel uses, on a
