@@ -9,14 +9,32 @@
 
 namespace matq {
 
+// One block per row.  Rows of D <= kHeld * 4 * 256 values with D % 4 == 0 are read once with
+// 16-byte loads and kept in registers between the sum of squares and the scaling; others take
+// two scalar passes.
+constexpr int kRmsHeld = 8;
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ h, int D, float eps,
                                                       __nv_bfloat16* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
   const int row = blockIdx.x;
   const float* hr = h + (size_t)row * D;
+  __nv_bfloat16* orow = out + (size_t)row * D;
+  const bool held = (D & 3) == 0 && D <= kRmsHeld * 4 * 256;
+  float4 v[kRmsHeld];
   float ss = 0.f;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) ss = fmaf(hr[i], hr[i], ss);
+  if (held) {
+#pragma unroll
+    for (int u = 0; u < kRmsHeld; ++u) {
+      const int i = threadIdx.x + u * 256;
+      v[u] = i < D / 4 ? reinterpret_cast<const float4*>(hr)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kRmsHeld; ++u)
+      ss = fmaf(v[u].x, v[u].x, fmaf(v[u].y, v[u].y, fmaf(v[u].z, v[u].z, fmaf(v[u].w, v[u].w, ss))));
+  } else {
+    for (int i = threadIdx.x; i < D; i += blockDim.x) ss = fmaf(hr[i], hr[i], ss);
+  }
   __shared__ float part[8];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -25,8 +43,22 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   float tot = 0.f;
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
   const float inv = rsqrtf(tot / (float)D + eps);
-  __nv_bfloat16* orow = out + (size_t)row * D;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) orow[i] = __float2bfloat16_rn(hr[i] * inv);
+  if (held) {
+#pragma unroll
+    for (int u = 0; u < kRmsHeld; ++u) {
+      const int i = threadIdx.x + u * 256;
+      if (i < D / 4) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(v[u].x * inv, v[u].y * inv);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(v[u].z * inv, v[u].w * inv);
+        uint2 o;
+        o.x = *reinterpret_cast<const uint32_t*>(&a);
+        o.y = *reinterpret_cast<const uint32_t*>(&b);
+        reinterpret_cast<uint2*>(orow)[i] = o;
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < D; i += blockDim.x) orow[i] = __float2bfloat16_rn(hr[i] * inv);
+  }
 }
 
 __device__ __forceinline__ float silu_f(float t) { return t / (1.0f + expf(-t)); }
