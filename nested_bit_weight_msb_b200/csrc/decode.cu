@@ -57,7 +57,8 @@ constexpr int kRowSlices = 4;        // warps split an item's row tiles four way
 // register budget of a thread stays at 255, and only two code variants share the I-cache)
 __host__ __device__ constexpr int k_slices(int NT) { return NT > 0 ? 2 : 2; }
 __host__ __device__ constexpr int dec_threads(int NT) { return 32 * kRowSlices * k_slices(NT); }
-// Resident CTAs per SM (CPS): two for M <= 8 and r in {2, 6, 8} on matrices with K <= 4096
+// Resident CTAs per SM (CPS): two for M <= 8 and r in {2, 6, 8}, and for M <= 16 and r in
+// {6, 8} (measured 12 % faster at r = 8), on matrices with K <= 4096
 // (each CTA's 8 warps then fit 128 registers a thread, so an SM runs 16 warps and hides more
 // latency: measured 7% faster at r = 2, the width with the shortest items; r = 6 and 8 carry
 // the most operand-building work per item), otherwise one.  On long-K matrices a row group
@@ -84,6 +85,8 @@ struct DecodeParams {
 template <int R, int NT, int GROUP, int CPS>
 struct DecodeLayout {
   static constexpr int RPW = rows_per_warp_tiles(R);
+  // the split-row-group slots (decode_workspace_bytes) hold 8 = CPS * RPW * NT fragments a lane
+  static_assert(CPS * RPW * NT <= 8, "partial-sum slots sized for CPS * RPW * NT <= 8");
   static constexpr int RG = kRowSlices * RPW;           // row tiles per item
   static constexpr int NG = kChunk / GROUP;             // groups per chunk
   static constexpr int NTOK = NT * 8;
@@ -692,7 +695,7 @@ template <int NT, int GROUP, int CPS>
 static cudaError_t launch_decode_r(int r, const uint8_t* planes, const PlaneGeom& g, const DecodeParams& P, int sms,
                                    cudaStream_t s) {
   switch (r) {
-    case 2: return launch_decode_t<2, NT, GROUP, CPS>(planes, g, P, sms, s);
+    case 2: return launch_decode_t<2, NT, GROUP, NT == 1 ? CPS : 1>(planes, g, P, sms, s);
     case 3: return launch_decode_t<3, NT, GROUP, 1>(planes, g, P, sms, s);
     case 4: return launch_decode_t<4, NT, GROUP, 1>(planes, g, P, sms, s);
     case 6: return launch_decode_t<6, NT, GROUP, CPS>(planes, g, P, sms, s);
@@ -728,6 +731,10 @@ cudaError_t launch_decode(const void* x, int M, int K, const void* planes, const
     return group == 64 ? launch_decode_r<1, 64, 2>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 2>(r, pl, g, P, sms, s);
   if (NT == 1)
     return group == 64 ? launch_decode_r<1, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<1, 128, 1>(r, pl, g, P, sms, s);
+  // M <= 16: two CTAs per SM on short-K matrices at r = 6 and 8 only (two row tiles a warp
+  // there; at r <= 4 four row tiles of two token tiles need more than 128 registers a thread)
+  if (g.KC <= 16 && r >= 6)
+    return group == 64 ? launch_decode_r<2, 64, 2>(r, pl, g, P, sms, s) : launch_decode_r<2, 128, 2>(r, pl, g, P, sms, s);
   return group == 64 ? launch_decode_r<2, 64, 1>(r, pl, g, P, sms, s) : launch_decode_r<2, 128, 1>(r, pl, g, P, sms, s);
 }
 
