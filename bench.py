@@ -621,7 +621,7 @@ _KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "common.cuh", "operands.cuh", "sync.cuh"),
 }
 NCU_TRAFFIC = {  # kernel kind -> capture (sources hash, launch it was taken on, bytes)
-    "decode": {"sha256": "6b013537a2205803101d7c90264281346a88460615dd1def453dd03e6a88ab45", "launch": "gate_up gated 28672x4096 r=2 M=1",
+    "decode": {"sha256": "7162c54c3875465eed93c3ec8e6ed433b6e04952f9c10aefd2bb17b1fdf2a84e", "launch": "gate_up gated 28672x4096 r=2 M=1",
                "bytes": 32_188_928 + 0},
     "prefill": {"sha256": "58199cae351b8d6212fb20b4465a2ca14b7fd9a967156d6ed4862827fef8cb53", "launch": "gate_up gated 28672x4096 r=4 M=2048",
                 "bytes": 78_321_664 + 30_037_760},
