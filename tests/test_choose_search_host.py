@@ -45,7 +45,7 @@ using std::isnan; using std::max; using std::min;
 namespace matq {
 """
 
-DRIVER = r"""
+HARNESS = r"""
 }  // namespace matq
 extern "C" void choose_host(const float* w, const float* s, const float* z, int n, int nw, const int* r,
                             const float* lam, int truncate, int force_scan, uint8_t* out) {
@@ -89,7 +89,7 @@ def search():
     cpp = os.path.join(BUILD, "choose_search_host.cpp")
     lib = os.path.join(BUILD, "libchoose_search_host.so")
     with open(cpp, "w") as f:
-        f.write(PRELUDE + _search_source() + DRIVER)
+        f.write(PRELUDE + _search_source() + HARNESS)
     subprocess.run([gxx, "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC",
                     "-o", lib, cpp], check=True)
     so = ctypes.CDLL(lib)

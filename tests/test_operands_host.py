@@ -57,7 +57,7 @@ inline uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }  // namespace matq
 """
 
-DRIVER = r"""
+HARNESS = r"""
 #include "operands.cuh"
 template <int R, int W>
 static void one(const matq::LaneWords& L, uint32_t* out) {
@@ -106,7 +106,7 @@ def build_host():
         f.write(COMMON_STUB)
     cpp = os.path.join(BUILD, "operands_host.cpp")
     with open(cpp, "w") as f:
-        f.write(DRIVER)
+        f.write(HARNESS)
     lib = os.path.join(BUILD, "liboperands_host.so")
     subprocess.run([gxx, "-O2", "-std=c++17", "-shared", "-fPIC", "-I", BUILD, "-o", lib, cpp], check=True)
     so = ctypes.CDLL(lib)
