@@ -199,12 +199,13 @@ def test_prefill_closed_forms(M):
     ((14336, 4096), 128, (2048,), (3, 4, 8)),
     ((4096, 14336), 128, (2048,), (3, 4, 8)),
     ((14336, 3584), 64, (32, 128, 512, 2048), (2, 3, 4, 6, 8)),
-    ((3584, 14336), 64, (32, 2048), (2, 8)),
+    ((3584, 14336), 64, (32, 128, 512, 2048), (2, 3, 4, 6, 8)),
 ])
 def test_prefill_full_size_sampled(M, shape, group, Ms, widths):
     """Benchmark shapes at the prefill batch sizes (8B FFN at M = 2048 with 1% outlier
-    channels x20; 9B FFN batch sweep), in the bench's launch configuration; 48 sampled output
-    rows against the oracle."""
+    channels x20; 9B FFN batch sweep at every width, the down projection through its K-split
+    path at M <= 512), in the bench's launch configuration; 48 sampled output rows against the
+    oracle."""
     import torch
     N, K = shape
     q, s, z = synth.parent_weights(N, K, group, seed=0, proj="gate" if N > K else "down")
