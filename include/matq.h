@@ -290,10 +290,12 @@ int matq_linear_rounded(const void* x, int M, int K,
  *               After the call completes on the device it holds 0, or the device-side
  *               wait-timeout code of this call (then y is undefined).
  *   no workspace arguments.
- * Limits: the sizes must fit the fixed scratch, i.e. matq_linear_workspace(M, K, N, group)
- * <= MATQ_NOALLOC_SCRATCH_BYTES; larger calls return MATQ_ESCRATCH and launch nothing.
- * Every M <= 16 (decode path) fits; M > 16 (prefill path) fits while 262,400 + M*K*2 bytes
- * (rounded up to 256) do, e.g. M <= 991 at K = 4096.  Use matq_linear with a caller workspace beyond that.
+ * Limits: the sizes must fit the fixed scratch: the smallest workspace matq_linear accepts for
+ * them (below) must be <= MATQ_NOALLOC_SCRATCH_BYTES; larger calls return MATQ_ESCRATCH and
+ * launch nothing.
+ * Every M <= 16 (decode path) fits; M > 16 (prefill path) fits while 262,400 + M*K*2 + M*4
+ * bytes (the last two each rounded up to 256) do, e.g. M <= 991 at K = 4096; such a call runs
+ * without K splits.  Use matq_linear with a caller workspace beyond that.
  * Set-up: the first call on each device, made with that device current, looks up the device
  * address of the array (cudaGetSymbolAddress; this can load libmatq's device code onto the
  * device) and caches it; a failure returns MATQ_ECUDA.  Make that first call before any
