@@ -397,15 +397,13 @@ __device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem,
               for (int nt = 0; nt < NT; ++nt)
                 __stcg(&mine[j * NT + nt], make_float4(yacc[j][nt][0], yacc[j][nt][1], yacc[j][nt][2], yacc[j][nt][3]));
           }
-          __threadfence();  // release: the partial sums before the ticket
-          __syncwarp();
+          __syncwarp();  // the warp's partial sums are stored before lane 0 takes the ticket
           int ticket = 0;
           if (lane == 0) {
-            ticket = atomicAdd(cnt, 1);
-            if (ticket == (int)(cl - cf)) {
-              __threadfence();  // acquire: every other contributor's partial sums (fence + ticket)
-              *reinterpret_cast<volatile int*>(cnt) = 0;  // leave the counter at zero for the next call
-            }
+            // acquire-release ticket: releases the warp's partial sums (cumulative through the
+            // warp barrier) and acquires every earlier contributor's
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(cnt) : "memory");
+            if (ticket == (int)(cl - cf)) *reinterpret_cast<volatile int*>(cnt) = 0;  // zero for the next call
           }
           ticket = __shfl_sync(0xffffffffu, ticket, 0);
           __syncwarp();  // orders the other lanes' loads after lane 0's acquire
