@@ -100,7 +100,12 @@ struct DecodeLayout {
   static constexpr int kStage = ((oZ + kMetaZ) + 127) & ~127;
   static constexpr int KSL = k_slices(NT);
   static constexpr int kThreads = dec_threads(NT);
-  static constexpr int kRed = (KSL - 1) * kRowSlices * RPW * NT * 4 * 32 * 4;
+  // k-slice reduction buffer: two of them at NT = 1, used by alternate flushes (the warps of
+  // k-slices > 0 then pass a flush without waiting for the k-slice-0 warps' stores and ticket;
+  // measured 1-3 % faster at M <= 8 and slower at M = 16)
+  static constexpr bool kTwoRed = NT == 1;
+  static constexpr int kRedHalf = (KSL - 1) * kRowSlices * RPW * NT * 4 * 32 * 4;
+  static constexpr int kRed = (kTwoRed ? 2 : 1) * kRedHalf;
   // ring depth: up to 4 stages within the CTA's share of the SM's shared memory
   static constexpr int kSmemBudget = CPS == 2 ? 113 * 1024 : 224 * 1024;
   static constexpr int kStagesFit = (kSmemBudget - kRed - 256) / kStage;
@@ -213,6 +218,7 @@ __device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem,
   const int rg_first = (int)(ib / P.KC);
   int rg = rg_first, kc = (int)(ib - (long long)rg_first * P.KC);
   int refills = 0;
+  int flushes = 0;  // flushes so far (selects the reduction buffer at NT = 1)
   for (int n = 0; n < nitems; ++n) {
     const int s = n % Lt::kStages;
     if (ok) ok = mbar_wait(&full[s], (n / Lt::kStages) & 1, P.err, 2);
@@ -316,11 +322,14 @@ __device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem,
     // flush at the end of a row group (or of this CTA's range); all warps get here for the
     // same items, so the four k-slices of a row slice meet at a named barrier
     if (n == nitems - 1 || kc == P.KC - 1) {
+      // With two buffers, flush f + 2 reuses flush f's only after every warp passed flush
+      // f + 1's barrier, which the k-slice-0 warps reach after reading flush f's sums.
+      float* redf = red + (Lt::kTwoRed ? (flushes++ & 1) * (Lt::kRedHalf / 4) : 0);
       const long long g0 = (long long)rg * P.KC, g1 = g0 + P.KC;
       const bool whole = g0 >= ib && g1 <= ie;
       if (KS > 0) {
         float4* mine =
-            reinterpret_cast<float4*>(red + ((KS - 1) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+            reinterpret_cast<float4*>(redf + ((KS - 1) * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
         for (int j = 0; j < RPW; ++j)
 #pragma unroll
@@ -331,7 +340,7 @@ __device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem,
       if (KS == 0) {
 #pragma unroll
         for (int k2 = 0; k2 < KSL - 1; ++k2) {
-          const float4* o = reinterpret_cast<const float4*>(red + (k2 * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
+          const float4* o = reinterpret_cast<const float4*>(redf + (k2 * kRowSlices + rs) * kSlotFloats + lane * kLaneFloats);
 #pragma unroll
           for (int j = 0; j < RPW; ++j)
 #pragma unroll
@@ -451,8 +460,8 @@ __device__ __forceinline__ int decode_warp(const DecodeParams& P, uint8_t* smem,
           }
         }
       }
-      // the reduction buffer may be overwritten only after the k-slice-0 warps have read it
-      asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
+      // one buffer: it may be overwritten only after the k-slice-0 warps have read it
+      if constexpr (!Lt::kTwoRed) asm volatile("bar.sync 1, %0;" ::"r"(Lt::kThreads) : "memory");
 #pragma unroll
       for (int j = 0; j < RPW; ++j)
 #pragma unroll
