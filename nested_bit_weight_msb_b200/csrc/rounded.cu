@@ -33,6 +33,7 @@ constexpr int kCorrThreads = 256;
 constexpr int kCorrWarps = kCorrThreads / 32;
 constexpr int kCorrSmem = 160 * 1024;   // activation window + block scales + sums
 constexpr int kCorrScaleBytes = 32 * 1024;
+constexpr int kSmemPerSM = 228 * 1024;   // shared memory of an SM
 
 struct CorrParams {
   const __nv_bfloat16* x;
@@ -228,24 +229,34 @@ __global__ void __launch_bounds__(kCorrThreads) overflow_correct_kernel(const __
   pdl_launch_dependents();
 }
 
-// Rows per CTA (even, so that gated row pairs stay together): enough CTAs for four per SM, at
-// least 16 rows, and the block's scales within kCorrScaleBytes.  Window: the rest of the
-// shared memory holds KW inputs x MP tokens of bf16 activations.
+// Rows per CTA (even, so that gated row pairs stay together): enough CTAs for one wave of as
+// many per SM as fit (four, fewer when the activation window is large: every CTA stages the
+// activations, so a CTA more per SM costs another copy of them), at least 16 rows, and the
+// block's scales within kCorrScaleBytes.  Window: the rest of the shared memory holds KW
+// inputs x MP tokens of bf16 activations.
 size_t overflow_correct_smem(int M, int K, int N, int G, int* rpc_out, int* kw_out) {
   const int MP = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
   const int sms = sm_count(current_device());
-  long long rpc = ((long long)N + 4LL * sms - 1) / (4LL * sms);
   const long long cap = kCorrScaleBytes / (2LL * G);
-  if (rpc > 512) rpc = 512;
-  if (rpc > cap) rpc = cap;
-  if (rpc < 16) rpc = 16;
-  rpc = (rpc + 1) & ~1LL;
-  const size_t fixed = (size_t)rpc * MP * 4 + ((size_t)rpc + 2) * 4 + (((size_t)rpc * G * 2 + 15) & ~size_t(15));
-  long long kw = (((long long)kCorrSmem - (long long)fixed) / (MP * 2)) & ~255LL;  // whole chunks
-  if (kw > K) kw = K;
+  long long rpc = 0, kw = 0;
+  size_t smem = 0;
+  auto layout = [&](long long per_sm) {
+    rpc = ((long long)N + per_sm * sms - 1) / (per_sm * sms);
+    if (rpc > 512) rpc = 512;
+    if (rpc > cap) rpc = cap;
+    if (rpc < 16) rpc = 16;
+    rpc = (rpc + 1) & ~1LL;
+    const size_t fixed = (size_t)rpc * MP * 4 + ((size_t)rpc + 2) * 4 + (((size_t)rpc * G * 2 + 15) & ~size_t(15));
+    kw = (((long long)kCorrSmem - (long long)fixed) / (MP * 2)) & ~255LL;  // whole chunks
+    if (kw > K) kw = K;
+    smem = fixed + (size_t)kw * MP * 2;
+  };
+  layout(4);
+  const long long fit = (long long)kSmemPerSM / (long long)(smem + 1024);  // + the runtime's reserve
+  if (fit < 4) layout(fit < 1 ? 1 : fit);
   if (rpc_out) *rpc_out = (int)rpc;
   if (kw_out) *kw_out = (int)kw;
-  return fixed + (size_t)kw * MP * 2;
+  return smem;
 }
 
 template <int MP>

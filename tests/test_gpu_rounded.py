@@ -178,3 +178,24 @@ def test_extra_precision_prefill_k_split(M):
     y = M.linear_rounded(dx, levels, r, ds, dz, N, G, row_ptr, cols, y_mode=M.MATQ_OUT_F32)
     check_close(y.cpu().numpy(), O.linear(xv.astype(np.float64), q, s, z, r, G, mode="extra_precision"),
                 what="extra precision K split")
+
+
+@pytest.mark.parametrize("Mt", [8, 16])
+@pytest.mark.parametrize("mode", ["bf16", "gated"])
+def test_extra_precision_long_k_windows(M, Mt, mode):
+    """A long input range (K = 14336, the 8B down projection's) at 8 and 16 tokens: the
+    correction stages the activations in two and three windows of inputs and walks the list once
+    per window; the decode path's dense part splits each row group across many CTAs."""
+    N, K, G, r = 264, 14336, 128, 2
+    q, s, z = _problem(N, K, G, seed=44, uniform=True)
+    levels, row_ptr, cols = extract(M, q, r, 3)
+    xb, xv = synth.activations(Mt, K, seed=6)
+    _, ds, dz, dx = to_device(q, s, z, xb)
+    ref = O.linear(xv.astype(np.float64), q, s, z, r, G, mode="extra_precision")
+    if mode == "bf16":
+        y = M.linear_rounded(dx, levels, r, ds, dz, N, G, row_ptr, cols)
+        check_close(y.float().cpu().numpy(), ref, what=f"long K M={Mt}")
+    else:
+        a = M.linear_rounded(dx, levels, r, ds, dz, N, G, row_ptr, cols, y_mode=M.MATQ_OUT_SILU_GATED)
+        check_close(a.float().cpu().numpy(), O.gated_product(ref[:, 0::2], ref[:, 1::2]),
+                    what=f"long K gated M={Mt}")
