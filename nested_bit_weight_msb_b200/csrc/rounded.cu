@@ -47,12 +47,45 @@ struct CorrParams {
   int y_mode;
 };
 
+// The MP staged activations of one input (MP consecutive bf16) as floats: one 16-byte load per
+// eight tokens, one 8- or 4-byte load below that.  The window is 16-byte aligned for MP >= 2
+// (the sums and row pointers before it fill whole 16-byte units), so every load is aligned.
+template <int MP>
+__device__ __forceinline__ void load_tokens(const __nv_bfloat16* xr, float (&xv)[MP]) {
+  if constexpr (MP == 1) {
+    xv[0] = __bfloat162float(xr[0]);
+  } else {
+    uint32_t u[MP / 2];
+    if constexpr (MP >= 8) {
+#pragma unroll
+      for (int v = 0; v < MP / 8; ++v) {
+        const uint4 q = reinterpret_cast<const uint4*>(xr)[v];
+        u[4 * v] = q.x;
+        u[4 * v + 1] = q.y;
+        u[4 * v + 2] = q.z;
+        u[4 * v + 3] = q.w;
+      }
+    } else if constexpr (MP == 4) {
+      const uint2 q = *reinterpret_cast<const uint2*>(xr);
+      u[0] = q.x;
+      u[1] = q.y;
+    } else {
+      u[0] = *reinterpret_cast<const uint32_t*>(xr);
+    }
+#pragma unroll
+    for (int i = 0; i < MP / 2; ++i) {
+      xv[2 * i] = __uint_as_float(u[i] << 16);  // bf16 is the high half of an fp32
+      xv[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+  }
+}
+
 template <int MP>
 __global__ void __launch_bounds__(kCorrThreads) overflow_correct_kernel(const __grid_constant__ CorrParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   float* acc = reinterpret_cast<float*>(smem);                          // [RPC][MP]
   int* rp = reinterpret_cast<int*>(acc + (size_t)P.RPC * MP);           // [RPC + 1] row pointers
-  uint16_t* sc = reinterpret_cast<uint16_t*>(rp + P.RPC + 2);           // [RPC][G] fp16 scales
+  uint16_t* sc = reinterpret_cast<uint16_t*>(rp + ((P.RPC + 5) & ~3));  // [RPC][G] fp16 scales
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(
       reinterpret_cast<uint8_t*>(sc) + (((size_t)P.RPC * P.G * 2 + 15) & ~size_t(15)));  // [KW][MP]
   const int tid = threadIdx.x;
@@ -178,9 +211,10 @@ __global__ void __launch_bounds__(kCorrThreads) overflow_correct_kernel(const __
         }
         if (k >= kw0 && k < kend) {
           const float w = __half2float(__ushort_as_half(sc[row * P.G + (k >> P.gshift)])) * P.step;
-          const __nv_bfloat16* xr = xs + (size_t)(k - kw0) * MP;
+          float xv[MP];
+          load_tokens<MP>(xs + (size_t)(k - kw0) * MP, xv);
 #pragma unroll
-          for (int m = 0; m < MP; ++m) a[m] = fmaf(w, __bfloat162float(xr[m]), a[m]);
+          for (int m = 0; m < MP; ++m) a[m] = fmaf(w, xv[m], a[m]);
         }
       }
       // end of the tile: the lanes' current rows are non-decreasing across the warp (a lane
@@ -246,7 +280,7 @@ size_t overflow_correct_smem(int M, int K, int N, int G, int* rpc_out, int* kw_o
     if (rpc > cap) rpc = cap;
     if (rpc < 16) rpc = 16;
     rpc = (rpc + 1) & ~1LL;
-    const size_t fixed = (size_t)rpc * MP * 4 + ((size_t)rpc + 2) * 4 + (((size_t)rpc * G * 2 + 15) & ~size_t(15));
+    const size_t fixed = (size_t)rpc * MP * 4 + (((size_t)rpc + 5) & ~size_t(3)) * 4 + (((size_t)rpc * G * 2 + 15) & ~size_t(15));
     kw = (((long long)kCorrSmem - (long long)fixed) / (MP * 2)) & ~255LL;  // whole chunks
     if (kw > K) kw = K;
     smem = fixed + (size_t)kw * MP * 2;
